@@ -1,0 +1,173 @@
+"""CPU oracle for the Qift W2A4 linear path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / reference leg of
+``bench.py`` may import this package.  The product path (``w2a4_gemm_b200``) never imports it
+and must fail loudly if its CUDA library is missing; there is no CPU fallback.
+
+The arithmetic lives in ``qift_oracle.c`` (plain C loops in IEEE binary32/binary64); this
+module only marshals numpy arrays.  The one step done here in numpy is the single rounding of
+the rotated activations to binary16 (``astype(np.float16)``, round-to-nearest-even), which the
+C code cannot express portably.  ``source_model`` holds the Gaussian level-set analysis.
+
+Paper: "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+Inference" (Huang, Tsai), Abstract.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+SET_QIFT, SET_POT, SET_STD = 0, 1, 2
+SET_NAMES = {"qift": SET_QIFT, "pot": SET_POT, "std": SET_STD}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        i64, i32, f32, f64, vp = C.c_int64, C.c_int32, C.c_float, C.c_double, C.c_void_p
+        L.qo_fwht_f64.argtypes = [vp, i64, i64, i32]
+        L.qo_rotate_f32.argtypes = [vp, i64, i64, i32]
+        L.qo_level.argtypes = [i32, i32]
+        L.qo_level.restype = i32
+        L.qo_candidate_scales.argtypes = [f32, i32, i32, f64, f64, vp]
+        L.qo_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
+        L.qo_unpack_codes.argtypes = [vp, i64, i64, vp]
+        L.qo_quantize_acts.argtypes = [vp, i64, i64, vp, vp]
+        L.qo_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, vp]
+        for name in ("qo_fwht_f64", "qo_rotate_f32", "qo_candidate_scales", "qo_quantize_weights",
+                     "qo_unpack_codes", "qo_quantize_acts", "qo_linear"):
+            getattr(L, name).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p) if a is not None else None
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} failed with code {rc}")
+
+
+def set_id(levelset) -> int:
+    return SET_NAMES[levelset] if isinstance(levelset, str) else int(levelset)
+
+
+# --------------------------------------------------------------------------------- rotation
+def fwht_f64(x: np.ndarray, block: int) -> np.ndarray:
+    """Block-diagonal normalised Sylvester Hadamard along the last axis, binary64 (R1, R2)."""
+    y = np.ascontiguousarray(x, dtype=np.float64).copy()
+    n = y.shape[-1]
+    _check(lib().qo_fwht_f64(_ptr(y), y.size // max(n, 1), n, block), "fwht_f64")
+    return y
+
+
+def rotate_f32(x: np.ndarray, block: int) -> np.ndarray:
+    """Same transform in binary32 with the canonical stage order (the weight rotation)."""
+    y = np.ascontiguousarray(x, dtype=np.float32).copy()
+    n = y.shape[-1]
+    _check(lib().qo_rotate_f32(_ptr(y), y.size // max(n, 1), n, block), "rotate_f32")
+    return y
+
+
+def rotate_f16(x: np.ndarray, block: int) -> np.ndarray:
+    """Activation rotation: binary16 in, binary32 stages, one rounding to binary16 out."""
+    assert x.dtype == np.float16
+    return rotate_f32(x.astype(np.float32), block).astype(np.float16)
+
+
+# ------------------------------------------------------------------------- weight quantizer
+def levels(levelset) -> np.ndarray:
+    s = set_id(levelset)
+    return np.array([lib().qo_level(s, c) for c in range(4)], dtype=np.int64)
+
+
+def candidate_scales(m: float, levelset, grid_points: int = 100, lo: float = 0.2, hi: float = 1.0):
+    out = np.zeros(grid_points, dtype=np.float32)
+    _check(lib().qo_candidate_scales(C.c_float(m), set_id(levelset), grid_points, lo, hi, _ptr(out)),
+           "candidate_scales")
+    return out
+
+
+def quantize_weights(w_rot: np.ndarray, levelset, grid_points: int = 100, lo: float = 0.2, hi: float = 1.0):
+    """Per-row MSE scale search + nearest-level encode + 2-bit pack.
+
+    Returns ``(codes u32 [N, K/16], scales f32 [N], row_mse f64 [N], best_k i32 [N])``.
+    """
+    w = np.ascontiguousarray(w_rot, dtype=np.float32)
+    n_out, n_in = w.shape
+    codes = np.zeros((n_out, n_in // 16), dtype=np.uint32)
+    scales = np.zeros(n_out, dtype=np.float32)
+    mse = np.zeros(n_out, dtype=np.float64)
+    best = np.zeros(n_out, dtype=np.int32)
+    _check(lib().qo_quantize_weights(_ptr(w), n_out, n_in, set_id(levelset), grid_points, lo, hi,
+                                      _ptr(codes), _ptr(scales), _ptr(mse), _ptr(best)), "quantize_weights")
+    return codes, scales, mse, best
+
+
+def unpack_codes(codes: np.ndarray, n_in: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    out = np.zeros((codes.shape[0], n_in), dtype=np.uint8)
+    _check(lib().qo_unpack_codes(_ptr(codes), codes.shape[0], n_in, _ptr(out)), "unpack_codes")
+    return out
+
+
+# --------------------------------------------------------------------- activation quantizer
+def quantize_acts(x: np.ndarray, block: int = 0):
+    """Rotate (if ``block``) and quantize activations to symmetric per-token INT4.
+
+    ``x`` is binary16 ``[T, K]``.  Returns ``(q int8 [T, K], s_a f32 [T], x_rot f16 [T, K])``.
+    """
+    assert x.dtype == np.float16
+    xr = rotate_f16(x, block) if block else x.copy()
+    xf = np.ascontiguousarray(xr.astype(np.float32))
+    T, K = xf.shape
+    q = np.zeros((T, K), dtype=np.int8)
+    s = np.zeros(T, dtype=np.float32)
+    _check(lib().qo_quantize_acts(_ptr(xf), T, K, _ptr(q), _ptr(s)), "quantize_acts")
+    return q, s, xr
+
+
+# ---------------------------------------------------------------------------------- linear
+def linear(q: np.ndarray, s_a: np.ndarray, codes: np.ndarray, s_w: np.ndarray, levelset,
+           out_dtype=np.float32):
+    """W2A4 linear: int32 accumulators and the binary32 epilogue (cast to ``out_dtype``).
+
+    Returns ``(y [T, N], acc int32 [T, N])``.
+    """
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    T, K = q.shape
+    N = codes.shape[0]
+    assert codes.shape[1] * 16 == K
+    acc = np.zeros((T, N), dtype=np.int32)
+    y = np.zeros((T, N), dtype=np.float32)
+    _check(lib().qo_linear(_ptr(q), _ptr(s_a), _ptr(codes), _ptr(s_w), set_id(levelset), T, N, K,
+                           _ptr(acc), _ptr(y)), "linear")
+    return y.astype(out_dtype), acc
+
+
+def pipeline(w: np.ndarray, x: np.ndarray, levelset, w_block: int, a_block: int, out_dtype=np.float16):
+    """Whole path: rotate W (binary32), quantize W, rotate+quantize x, W2A4 linear."""
+    w_rot = rotate_f32(w, w_block)
+    codes, s_w, mse, best = quantize_weights(w_rot, levelset)
+    q, s_a, _ = quantize_acts(x, a_block)
+    y, acc = linear(q, s_a, codes, s_w, levelset, out_dtype)
+    return dict(w_rot=w_rot, codes=codes, s_w=s_w, row_mse=mse, best_k=best, q=q, s_a=s_a, y=y, acc=acc)
+
+
+def threads() -> int:
+    """Host threads the oracle's OpenMP loops use."""
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v else (os.cpu_count() or 1)
