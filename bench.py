@@ -1,0 +1,407 @@
+"""Benchmark of the Qift W2A4 linear path on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|decode16|prefill|single]
+
+Workloads (synthetic, seeded; shapes of LLaMA linear modules):
+  decode   (default) LLaMA-7B q_proj 4096x4096, 1 token, 4096-point Hadamard, Qift {+-1,+-3}
+  decode16 LLaMA-3.1-8B MLP (gate/up 14336x4096, down 4096x14336), 16 tokens, 128-block, PoT
+  prefill  LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008), 2048 tokens, 128-block, Qift
+  single   one 256x512 linear, 8 tokens (parity case; timed for completeness)
+
+A step is one online forward pass over one batch: qift_quantize_acts (rotation + INT4) and
+qift_linear for every linear of the workload.  The weights are quantized once, offline
+(qift_rotate + qift_quantize_weights), and are resident in HBM; those two offline stages are
+timed in the same run and reported under "stages".  Decode workloads cycle through enough
+distinct weight copies that every step streams its codes from HBM, not L2.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W2A4 Qift linear: decode GB/s & prefill TOPS, % of B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    """HBM GB/s and int8 dense TOPS (burst, sustained) from the measured peak file."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    src = "measured"
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        hbm, bf16, bf16s = p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        hbm, bf16, bf16s, src = 6650.0, 1590.0, 1400.0, "fallback"
+    # int8 dense = bf16 dense x 2 (nominal 4.5 vs 2.25 PFLOP/s per GPU).
+    return dict(hbm_gbs=hbm, int8_tops=2.0 * bf16, int8_tops_sustained=2.0 * bf16s, source=src)
+
+
+# ----------------------------------------------------------------------------- workloads
+def workload_def(name):
+    from w2a4_gemm_b200 import synth
+    return {"decode": synth.LLAMA7B_QPROJ_DECODE, "decode16": synth.LLAMA31_8B_MLP_DECODE16,
+            "prefill": synth.LLAMA7B_MLP_PREFILL, "single": synth.SINGLE_256x512}[name]
+
+
+def linear_bytes(T, N, K, out_bytes):
+    """Algorithmic HBM bytes of one qift_linear: codes + w scales + int8 acts + act scales + y."""
+    return N * K // 4 + 4 * N + T * K + 4 * T + T * N * out_bytes
+
+
+def acts_bytes(T, K):
+    """Algorithmic HBM bytes of one qift_quantize_acts: fp16 in, int8 + scale out."""
+    return 2 * T * K + T * K + 4 * T
+
+
+# ------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                p = [x.strip() for x in ln.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()) if rows else None,
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- our path
+class OursState:
+    """Device-resident inputs of one workload: quantized weight copies and activation slots."""
+
+    def __init__(self, wl, torch, qg, copies):
+        self.wl, self.torch, self.qg = wl, torch, qg
+        dev = torch.device("cuda")
+        self.out_dt = torch.float16 if wl.out_dtype == "f16" else torch.float32
+        self.layers = []
+        self.offline = []
+        for lin in wl.linears:
+            W = torch.from_numpy(wl.w(lin)).to(dev)
+            w_rot = qg.qift_rotate(W, wl.w_block)
+            codes, s_w, _ = qg.qift_quantize_weights(w_rot, wl.levelset, with_mse=False)
+            self.offline.append((W, lin))
+            cc = [codes] + [codes.clone() for _ in range(copies - 1)]
+            sc = [s_w] + [s_w.clone() for _ in range(copies - 1)]
+            xs = [torch.from_numpy(wl.x(lin)).to(dev) for _ in range(1)]
+            xs = xs + [xs[0].clone() for _ in range(copies - 1)]
+            T, K, N = wl.tokens, lin.n_in, lin.n_out
+            q = [torch.empty((T, K), dtype=torch.int8, device=dev) for _ in range(copies)]
+            sa = [torch.empty(T, dtype=torch.float32, device=dev) for _ in range(copies)]
+            y = [torch.empty((T, N), dtype=self.out_dt, device=dev) for _ in range(copies)]
+            self.layers.append(dict(lin=lin, codes=cc, s_w=sc, x=xs, q=q, sa=sa, y=y))
+        self.copies = copies
+
+    def step(self, i):
+        qg, wl = self.qg, self.wl
+        c = i % self.copies
+        for L in self.layers:
+            qg.qift_quantize_acts(L["x"][c], wl.a_block, out_q=L["q"][c], out_scales=L["sa"][c])
+            qg.qift_linear(L["q"][c], L["sa"][c], L["codes"][c], L["s_w"][c], wl.levelset, self.out_dt,
+                           out=L["y"][c])
+
+    def launches_per_step(self):
+        return 2 * len(self.layers)
+
+
+def time_region(torch, fn, iters):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for i in range(iters):
+        fn(i)
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / 1e3  # seconds
+
+
+def run_ours(args, rank, world):
+    import torch
+    import w2a4_gemm_b200 as qg
+    from w2a4_gemm_b200 import build
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    build.build()
+    qg.lib()
+    torch.cuda.set_device(rank % torch.cuda.device_count())
+    wl = workload_def(args.workload)
+    pk = peaks()
+    T = wl.tokens
+    wbytes = sum(l.n_out * l.n_in // 4 for l in wl.linears)
+    copies = max(1, min(64, int(np.ceil(3 * L2_BYTES / max(wbytes, 1))))) if T <= 16 else 1
+    st = OursState(wl, torch, qg, copies)
+    out_b = 2 if wl.out_dtype == "f16" else 4
+    step_bytes = sum(linear_bytes(T, l.n_out, l.n_in, out_b) for l in wl.linears)
+    step_ops = sum(2 * T * l.n_out * l.n_in for l in wl.linears)
+    decode = T <= 16
+
+    for i in range(args.warmup):
+        st.step(i)
+    torch.cuda.synchronize()
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        secs = time_region(torch, st.step, args.steps)
+        if world > 1:
+            t = torch.tensor([secs], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            secs = float(t.item())
+    clocks = clk.summary()
+
+    # Per-kernel live timing over the same cycled inputs (one kernel type per loop).
+    L0 = st.layers[0]
+    lin0 = L0["lin"]
+    reps = max(20, args.steps)
+    t_acts = time_region(torch, lambda i: qg.qift_quantize_acts(L0["x"][i % copies], wl.a_block,
+                                                                out_q=L0["q"][i % copies],
+                                                                out_scales=L0["sa"][i % copies]), reps) / reps
+    t_lin = time_region(torch, lambda i: qg.qift_linear(L0["q"][i % copies], L0["sa"][i % copies],
+                                                        L0["codes"][i % copies], L0["s_w"][i % copies], wl.levelset,
+                                                        st.out_dt, out=L0["y"][i % copies]), reps) / reps
+    W, _ = st.offline[0]
+    w_rot = torch.empty_like(W)
+    t_rot = time_region(torch, lambda i: qg.qift_rotate(W, wl.w_block, out=w_rot), 5) / 5
+    t_qw = time_region(torch, lambda i: qg.qift_quantize_weights(w_rot, wl.levelset, with_mse=False), 2) / 2
+
+    N0, K0 = lin0.n_out, lin0.n_in
+    lin_b = linear_bytes(T, N0, K0, out_b)
+    act_b = acts_bytes(T, K0)
+    rot_b = 8 * N0 * K0
+    stages = {
+        "a1_rotate_weights": {"ms": t_rot * 1e3, "bytes": rot_b, "GB/s": rot_b / t_rot / 1e9,
+                              "frac_hbm": rot_b / t_rot / 1e9 / pk["hbm_gbs"], "bound": "hbm"},
+        "a2_quantize_weights": {"ms": t_qw * 1e3, "weights_per_s": N0 * K0 / t_qw,
+                                "candidate_evals_per_s": N0 * K0 * 100 / t_qw, "bound": "alu"},
+        "a3a4_quantize_acts": {"ms": t_acts * 1e3, "bytes": act_b, "GB/s": act_b / t_acts / 1e9,
+                               "frac_hbm": act_b / t_acts / 1e9 / pk["hbm_gbs"], "bound": "hbm"},
+        "a5_linear": {"ms": t_lin * 1e3, "bytes": lin_b, "GB/s": lin_b / t_lin / 1e9,
+                      "TOPS": 2 * T * N0 * K0 / t_lin / 1e12,
+                      "frac_hbm": lin_b / t_lin / 1e9 / pk["hbm_gbs"],
+                      "frac_int8": 2 * T * N0 * K0 / t_lin / 1e12 / pk["int8_tops"]},
+    }
+
+    if decode:
+        value = world * step_bytes * args.steps / secs / 1e9
+        unit = "GB/s"
+        roof = {"bound": "hbm", "achieved": lin_b / t_lin / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": lin_b / t_lin / 1e9 / pk["hbm_gbs"], "traffic": None, "kernel": "qift_linear (GEMV)",
+                "peak_source": pk["source"] + " copy bandwidth, burst"}
+    else:
+        value = world * step_ops * args.steps / secs / 1e12
+        unit = "TOPS"
+        ach = 2 * T * N0 * K0 / t_lin / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk["int8_tops"], "unit": "TOPS",
+                "frac": ach / pk["int8_tops"], "traffic": None, "kernel": "qift_linear (GEMM)",
+                "peak_source": pk["source"] + " bf16 burst x 2 (int8 nominal ratio)"}
+
+    # End to end through the public API: pinned host x -> device, both calls, y -> pinned host.
+    hx = [torch.from_numpy(wl.x(L["lin"])).pin_memory() for L in st.layers]
+    hy = [torch.empty((T, L["lin"].n_out), dtype=st.out_dt).pin_memory() for L in st.layers]
+
+    def e2e_step(i):
+        c = i % copies
+        for j, L in enumerate(st.layers):
+            L["x"][c].copy_(hx[j], non_blocking=True)
+            qg.qift_quantize_acts(L["x"][c], wl.a_block, out_q=L["q"][c], out_scales=L["sa"][c])
+            qg.qift_linear(L["q"][c], L["sa"][c], L["codes"][c], L["s_w"][c], wl.levelset, st.out_dt,
+                           out=L["y"][c])
+            hy[j].copy_(L["y"][c], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    e2e_secs = time_region(torch, e2e_step, args.steps)
+    if world > 1:
+        t = torch.tensor([e2e_secs], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_secs = float(t.item())
+    h2d = sum(x.numel() * x.element_size() for x in hx)
+    d2h = sum(y.numel() * y.element_size() for y in hy)
+    e2e_val = world * (step_bytes if decode else step_ops) * args.steps / e2e_secs / (1e9 if decode else 1e12)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "tokens": T,
+                   "linears": [[l.name, l.n_out, l.n_in] for l in wl.linears], "levelset": wl.levelset,
+                   "hadamard_block": wl.a_block, "out_dtype": wl.out_dtype,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": (f"inputs larger than L2: {copies} weight copies ({copies * wbytes / 1e6:.0f} MB codes) "
+                          "cycled step to step") if decode else "inputs larger than L2 (activations + outputs)",
+                   "step": "qift_quantize_acts + qift_linear per linear; weights quantized offline"},
+        "roofline": roof, "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d,
+                                  "d2h_bytes_per_step": d2h},
+        "gpu_launches": st.launches_per_step() * args.steps, "clocks": clocks, "stages": stages,
+    }
+    return line
+
+
+# ------------------------------------------------------------------------- CPU oracle arm
+def oracle_step_fn(wl, sample_tokens):
+    """Returns (step callable, bytes or ops per step, description) for the CPU oracle."""
+    import oracle
+    prepared = []
+    for lin in wl.linears:
+        W = wl.w(lin)
+        codes, s_w, _, _ = oracle.quantize_weights(oracle.rotate_f32(W, wl.w_block), wl.levelset)
+        x = wl.x(lin)[:sample_tokens]
+        prepared.append((lin, codes, s_w, x))
+
+    def step():
+        for lin, codes, s_w, x in prepared:
+            q, sa, _ = oracle.quantize_acts(x, wl.a_block)
+            oracle.linear(q, sa, codes, s_w, wl.levelset, np.float16)
+
+    return step, prepared
+
+
+def run_cpu(wl, budget_s, sample_tokens):
+    import oracle
+    step, prepared = oracle_step_fn(wl, sample_tokens)
+    step()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        step()
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    secs = (time.perf_counter() - t0) / n
+    T = sample_tokens
+    out_b = 2
+    by = sum(linear_bytes(T, l.n_out, l.n_in, out_b) for l, *_ in prepared)
+    ops = sum(2 * T * l.n_out * l.n_in for l, *_ in prepared)
+    return secs, by, ops, oracle.threads(), n
+
+
+def cpu_baseline_obj(wl, budget_s=10.0):
+    T = 1
+    secs, by, ops, cores, n = run_cpu(wl, budget_s, T)
+    decode = wl.tokens <= 16
+    val = by / secs / 1e9 if decode else ops / secs / 1e12
+    return {"value": val, "unit": "GB/s" if decode else "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{n} oracle steps of {T} token(s) over all linears of the workload "
+                      f"(quantize_acts + linear in plain C); {secs * 1e3:.1f} ms per step"}
+
+
+def run_reference(args):
+    # The oracle as it stands, one token per step (a bounded sample of the workload).
+    wl = workload_def(args.workload)
+    T = 1
+    decode = wl.tokens <= 16
+    step, prepared = oracle_step_fn(wl, T)
+    for _ in range(min(args.warmup, 3)):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    secs = (time.perf_counter() - t0)
+    by = sum(linear_bytes(T, l.n_out, l.n_in, 2) for l, *_ in prepared)
+    ops = sum(2 * T * l.n_out * l.n_in for l, *_ in prepared)
+    val = (by if decode else ops) * args.steps / secs / (1e9 if decode else 1e12)
+    unit = "GB/s" if decode else "TOPS"
+    import oracle
+    return {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "config": {"workload": wl.name, "tokens_per_step": T},
+            "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"{args.steps} oracle steps of {T} token(s)"},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single"], default="decode")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)))
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    line = run_ours(args, rank, world)
+    if rank == 0:
+        line["cpu_baseline"] = cpu_baseline_obj(workload_def(args.workload), args.cpu_budget) if world == 1 else None
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+"""GPU-vs-oracle parity of every stage of the Qift W2A4 path, called through the C ABI.
+
+Integer outputs (packed codes, INT4 activations, the int32 accumulators behind y) must match
+bit for bit.  Floating-point outputs are checked against the tolerances of the contract --
+fp32 epilogue |g - r| <= 1e-5 |r| + 1e-5 rms(r), fp16 rotation <= 2e-3 |r| + 2e-3 rms(r) --
+and, because both sides run the same IEEE operations in the same order, also for exact
+equality.  Inputs come from the seeded generators both sides share; expected values come from
+the CPU oracle only.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w2a4_gemm_b200 as qg
+from w2a4_gemm_b200 import build, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    qg.lib()
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def tol_check(got, ref, rel):
+    got = got.astype(np.float64)
+    ref = ref.astype(np.float64)
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    bad = np.abs(got - ref) > rel * np.abs(ref) + rel * rms
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside tolerance; max err {np.abs(got - ref).max()}"
+
+
+def codes_u32(t):
+    return host(t).view(np.uint32)
+
+
+# ------------------------------------------------------------------------------ rotation
+@pytest.mark.parametrize("block", [2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096])
+def test_rotate_f32_parity(block):
+    rows = 37
+    n = max(block, 4096) if block >= 1024 else block * 24
+    w = synth.weights(rows, n, (block, 1))
+    ref = oracle.rotate_f32(w, block)
+    got = host(qg.qift_rotate(dev(w), block))
+    tol_check(got, ref, 2e-3)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("block", [2, 16, 128, 512, 2048, 4096])
+def test_rotate_f16_parity(block):
+    x = synth.activations(19, max(block, 256) * 3, (block, 2), n_outliers=5)
+    ref = oracle.rotate_f16(x, block)
+    got = host(qg.qift_rotate(dev(x), block))
+    tol_check(got, ref, 2e-3)
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
+def test_rotate_in_place():
+    w = synth.weights(8, 4096, (5,))
+    t = dev(w)
+    qg.qift_rotate(t, 4096, out=t)
+    assert np.array_equal(host(t).view(np.uint32), oracle.rotate_f32(w, 4096).view(np.uint32))
+
+
+# ------------------------------------------------------------------------ weight quantizer
+@pytest.mark.parametrize("name", ["qift", "pot", "std"])
+@pytest.mark.parametrize("n_out,n_in,block", [(5, 16, 16), (33, 48, 16), (64, 512, 128), (40, 4096, 4096),
+                                               (9, 11008, 128)])
+def test_quantize_weights_parity(name, n_out, n_in, block):
+    w = oracle.rotate_f32(synth.weights(n_out, n_in, (n_in, 3)), block)
+    codes, scales, mse, best = oracle.quantize_weights(w, name)
+    gc, gs, gm = qg.qift_quantize_weights(dev(w), name)
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+    assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
+def test_quantize_weights_edge_rows():
+    # all-zero row, a single huge outlier, -0.0 entries, exact midpoints, constant row
+    K = 64
+    w = np.zeros((6, K), np.float32)
+    w[1, 7] = 1e3
+    w[1, 8:] = 1e-3
+    w[2, :] = -0.0
+    w[2, 3] = 0.5
+    w[3, :] = np.float32(0.25)
+    w[4, ::2] = np.float32(0.75)
+    w[4, 1::2] = np.float32(-0.25)
+    w[5] = synth.weights(1, K, (99,))[0]
+    for name in ("qift", "pot", "std"):
+        for grid, lo, hi in ((100, 0.2, 1.0), (2, 1.0, 1.0), (256, 0.05, 4.0)):
+            codes, scales, mse, _ = oracle.quantize_weights(w, name, grid, lo, hi)
+            gc, gs, gm = qg.qift_quantize_weights(dev(w), name, grid, lo, hi)
+            assert np.array_equal(codes_u32(gc), codes), (name, grid)
+            assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+            assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
+# -------------------------------------------------------------------- activation quantizer
+@pytest.mark.parametrize("block", [0, 16, 128, 512, 4096])
+@pytest.mark.parametrize("T,K", [(1, 4096), (3, 512), (16, 11008), (33, 4096)])
+def test_quantize_acts_parity(block, T, K):
+    if block and K % block:
+        pytest.skip("block must divide K")
+    x = synth.activations(T, K, (T, K), n_outliers=synth.outlier_count(K))
+    q, s, _ = oracle.quantize_acts(x, block)
+    gq, gs = qg.qift_quantize_acts(dev(x), block)
+    assert np.array_equal(host(gq), q)
+    assert np.array_equal(host(gs).view(np.uint32), s.view(np.uint32))
+
+
+def test_quantize_acts_zero_and_tiny_tokens():
+    x = np.zeros((4, 256), np.float16)
+    x[1, 5] = np.float16(-0.0)
+    x[2, 17] = np.float16(6e-8)          # subnormal fp16
+    x[3] = synth.activations(1, 256, (7,))[0]
+    for block in (0, 256, 64):
+        q, s, _ = oracle.quantize_acts(x, block)
+        gq, gs = qg.qift_quantize_acts(dev(x), block)
+        assert np.array_equal(host(gq), q)
+        assert np.array_equal(host(gs).view(np.uint32), s.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------------- linear
+def _linear_case(name, T, N, K, seed, out_dtype):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-7, 8, size=(T, K)).astype(np.int8)
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 16), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    s_a = rng.uniform(0.1, 2.0, T).astype(np.float32)
+    npdt = np.float16 if out_dtype == torch.float16 else np.float32
+    y, _ = oracle.linear(q, s_a, codes, s_w, name, npdt)
+    gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), name, out_dtype)
+    return host(gy), y
+
+
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("T,N,K", [(1, 1, 16), (1, 4096, 4096), (1, 37, 48), (2, 33, 528), (3, 70, 1024),
+                                    (5, 17, 4096), (16, 129, 4096), (16, 64, 14336), (33, 40, 64)])
+def test_linear_parity(name, T, N, K):
+    for out_dtype in (torch.float32, torch.float16):
+        got, ref = _linear_case(name, T, N, K, T * 1000 + N + K, out_dtype)
+        tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
+        assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
+                              ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32))
+
+
+def test_linear_extreme_accumulators():
+    # Every activation +-7 and every weight at the outer level: |acc| = 7 * 4 * K at K = 32768.
+    T, N, K = 2, 8, 32768
+    q = np.full((T, K), 7, np.int8)
+    q[1] = -7
+    codes = np.full((N, K // 16), 0xFFFFFFFF, np.uint32)   # code 3 everywhere
+    codes[1::2] = 0                                         # code 0 everywhere
+    s_w = np.full(N, 1.0, np.float32)
+    s_a = np.full(T, 1.0, np.float32)
+    for name, top in (("qift", 3), ("pot", 4)):
+        y, acc = oracle.linear(q, s_a, codes, s_w, name, np.float32)
+        assert np.abs(acc).max() == 7 * top * K
+        gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), name, torch.float32)
+        assert np.array_equal(host(gy), y)
+
+
+# ---------------------------------------------------------------------- whole path, small
+def test_single_linear_256x512_end_to_end():
+    wl = synth.SINGLE_256x512
+    lin = wl.linears[0]
+    W, x = wl.w(lin), wl.x(lin)
+    ref = oracle.pipeline(W, x, wl.levelset, wl.w_block, wl.a_block, out_dtype=np.float32)
+    w_rot = qg.qift_rotate(dev(W), wl.w_block)
+    gc, gs, gm = qg.qift_quantize_weights(w_rot, wl.levelset)
+    gq, gsa = qg.qift_quantize_acts(dev(x), wl.a_block)
+    gy = qg.qift_linear(gq, gsa, gc, gs, wl.levelset, torch.float32)
+    assert np.array_equal(host(w_rot).view(np.uint32), ref["w_rot"].view(np.uint32))
+    assert np.array_equal(codes_u32(gc), ref["codes"])
+    assert np.array_equal(host(gq), ref["q"])
+    tol_check(host(gy), ref["y"], 1e-5)
+    assert np.array_equal(host(gy), ref["y"])

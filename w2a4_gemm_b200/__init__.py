@@ -1,0 +1,159 @@
+"""Python binding of libqift.so -- the B200 (sm_100a) hot path of Qift W2A4 linear layers.
+
+"Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+Inference" (Huang, Tsai), Abstract: Hadamard-rotated weights and activations, fixed no-zero
+2-bit level sets with one scale per output channel, 4-bit activations.
+
+The functions here carry the C ABI's names (``include/qift.h``) and only marshal arguments:
+they check devices, dtypes and shapes, allocate outputs with torch, and pass raw device
+pointers plus the current CUDA stream to the library.  Every step of the path runs in the
+library's kernels.  There is no CPU fallback: without the built library or a CUDA device
+these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqift.so")
+
+QIFT_OK, QIFT_ERR_INVALID_ARG, QIFT_ERR_UNSUPPORTED, QIFT_ERR_CUDA, QIFT_ERR_TIMEOUT = range(5)
+QIFT_SET_QIFT, QIFT_SET_POT, QIFT_SET_STD = 0, 1, 2
+QIFT_F32, QIFT_F16 = 0, 1
+LEVELSETS = {"qift": QIFT_SET_QIFT, "pot": QIFT_SET_POT, "std": QIFT_SET_STD}
+
+_lib = None
+
+
+class QiftError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {qift_status_string(status)}")
+
+
+def lib() -> C.CDLL:
+    """Load libqift.so from the package directory; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m w2a4_gemm_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        i64, i32, f64, vp = C.c_int64, C.c_int32, C.c_double, C.c_void_p
+        L.qift_rotate.argtypes = [vp, vp, i32, i64, i64, i32, vp]
+        L.qift_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
+        L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+        L.qift_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, i32, vp]
+        L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
+        L.qift_status_string.argtypes = [i32]
+        L.qift_status_string.restype = C.c_char_p
+        for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear",
+                     "qift_device_error"):
+            getattr(L, name).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def qift_status_string(status: int) -> str:
+    return lib().qift_status_string(int(status)).decode()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _check(status: int, what: str):
+    if status != QIFT_OK:
+        raise QiftError(status, what)
+
+
+def _set(levelset) -> int:
+    return LEVELSETS[levelset] if isinstance(levelset, str) else int(levelset)
+
+
+def qift_rotate(x: torch.Tensor, block: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Block-diagonal normalised Walsh-Hadamard rotation along the last axis (fp32 or fp16)."""
+    _cuda(x, "x")
+    if x.dtype not in (torch.float32, torch.float16):
+        raise ValueError("x must be float32 or float16")
+    y = torch.empty_like(x) if out is None else _cuda(out, "out", x.dtype)
+    n = x.shape[-1]
+    rows = x.numel() // n if n else 0
+    dt = QIFT_F32 if x.dtype == torch.float32 else QIFT_F16
+    _check(lib().qift_rotate(_ptr(x), _ptr(y), dt, rows, n, block, _stream(stream)), "qift_rotate")
+    return y
+
+
+def qift_quantize_weights(w_rot: torch.Tensor, levelset="qift", grid_points: int = 100, lo: float = 0.2,
+                          hi: float = 1.0, with_mse: bool = True, stream=None):
+    """Per-row scale search + nearest-level encode + 2-bit pack.
+
+    Returns ``(codes int32-viewed-as-u32 [N, K/16], scales f32 [N], row_mse f64 [N] or None)``.
+    """
+    _cuda(w_rot, "w_rot", torch.float32)
+    n_out, n_in = w_rot.shape
+    dev = w_rot.device
+    codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
+    scales = torch.empty(n_out, dtype=torch.float32, device=dev)
+    mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
+    _check(lib().qift_quantize_weights(_ptr(w_rot), n_out, n_in, _set(levelset), grid_points, lo, hi,
+                                       _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
+           "qift_quantize_weights")
+    return codes, scales, mse
+
+
+def qift_quantize_acts(x: torch.Tensor, block: int = 0, out_q: torch.Tensor | None = None,
+                       out_scales: torch.Tensor | None = None, stream=None):
+    """Optional rotation + symmetric per-token INT4.  Returns ``(q int8 [T, K], s_a f32 [T])``."""
+    _cuda(x, "x", torch.float16)
+    T, K = x.shape
+    q = torch.empty((T, K), dtype=torch.int8, device=x.device) if out_q is None else _cuda(out_q, "out_q", torch.int8)
+    s = torch.empty(T, dtype=torch.float32, device=x.device) if out_scales is None else \
+        _cuda(out_scales, "out_scales", torch.float32)
+    _check(lib().qift_quantize_acts(_ptr(x), T, K, block, _ptr(q), _ptr(s), _stream(stream)), "qift_quantize_acts")
+    return q, s
+
+
+def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w_scale: torch.Tensor,
+                levelset="qift", out_dtype=torch.float16, out: torch.Tensor | None = None, stream=None):
+    """Fused W2A4 linear: ``y[t, n] = ((float)acc * w_scale[n]) * act_scale[t]``."""
+    _cuda(q, "q", torch.int8)
+    _cuda(act_scale, "act_scale", torch.float32)
+    _cuda(codes, "codes")
+    _cuda(w_scale, "w_scale", torch.float32)
+    if codes.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("codes must be 32-bit words")
+    T, K = q.shape
+    N = codes.shape[0]
+    if codes.shape[1] * 16 != K:
+        raise ValueError("codes must be [n_out, n_in/16]")
+    y = torch.empty((T, N), dtype=out_dtype, device=q.device) if out is None else _cuda(out, "out", out_dtype)
+    dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
+    _check(lib().qift_linear(_ptr(q), _ptr(act_scale), _ptr(codes), _ptr(w_scale), _set(levelset), T, N, K,
+                             _ptr(y), dt, _stream(stream)), "qift_linear")
+    return y
+
+
+def qift_device_error(stream=None) -> tuple[int, int]:
+    """Synchronise the stream, read and clear the device error word: ``(status, raw word)``."""
+    detail = C.c_int32(0)
+    st = lib().qift_device_error(_stream(stream), C.byref(detail))
+    return st, detail.value

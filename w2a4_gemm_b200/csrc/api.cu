@@ -1,0 +1,104 @@
+// api.cu -- the extern "C" entry points of libqift.so: host-side validation and dispatch.
+// Declarations, argument meaning, layouts and error behaviour are documented in qift.h.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/qift.h"
+#include "internal.h"
+
+namespace {
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+constexpr int64_t kMaxInner = 32768;  // keeps |acc| < 2^24 and a token / row in shared memory
+
+qift_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QIFT_OK : QIFT_ERR_CUDA; }
+
+bool valid_block(int64_t b) { return is_pow2(b) && b >= 2 && b <= 4096; }
+
+}  // namespace
+
+extern "C" {
+
+qift_status qift_rotate(const void* x, void* y, qift_dtype dt, int64_t rows, int64_t n, int32_t block,
+                        void* stream) {
+    if (dt != QIFT_F32 && dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
+    if (rows < 0 || n < 0 || !valid_block(block) || n % block != 0) return QIFT_ERR_INVALID_ARG;
+    if (rows == 0 || n == 0) return QIFT_OK;
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return QIFT_ERR_INVALID_ARG;
+    const int64_t esz = dt == QIFT_F32 ? 4 : 2;
+    if (rows > INT64_MAX / n / esz) return QIFT_ERR_INVALID_ARG;
+    const uintptr_t bytes = (uintptr_t)(rows * n * esz);
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+    if (xa != ya && xa < ya + bytes && ya < xa + bytes) return QIFT_ERR_INVALID_ARG;  // partial overlap
+    return from_cuda(qift::launch_rotate(x, y, dt == QIFT_F16, rows, n, block, static_cast<cudaStream_t>(stream)));
+}
+
+qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_in, qift_levelset set,
+                                  int32_t grid_points, double lo, double hi, uint32_t* codes, float* scales,
+                                  double* row_mse, void* stream) {
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (grid_points < 2 || grid_points > 256) return QIFT_ERR_INVALID_ARG;
+    if (!(lo > 0.0) || !(hi >= lo) || !(hi <= 4.0)) return QIFT_ERR_INVALID_ARG;
+    if (n_in > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (n_out == 0) return QIFT_OK;
+    if (!w_rot || !codes || !scales || !aligned16(w_rot) || !aligned16(codes) || !aligned4(scales))
+        return QIFT_ERR_INVALID_ARG;
+    if (row_mse && !aligned8(row_mse)) return QIFT_ERR_INVALID_ARG;
+    if (n_out > 0x7fffffff) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(qift::launch_quantize_weights(w_rot, n_out, n_in, (int)set, grid_points, lo, hi, codes, scales,
+                                                   row_mse, static_cast<cudaStream_t>(stream)));
+}
+
+qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int32_t block, int8_t* q,
+                               float* scales, void* stream) {
+    if (tokens < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (block != 0 && (!valid_block(block) || n_in % block != 0)) return QIFT_ERR_INVALID_ARG;
+    if (n_in > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (tokens == 0) return QIFT_OK;
+    if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || !aligned4(scales)) return QIFT_ERR_INVALID_ARG;
+    if (tokens > 0x7fffffff) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(
+        qift::launch_quantize_acts(x, tokens, n_in, block, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint32_t* codes, const float* w_scale,
+                        qift_levelset set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, qift_dtype out_dt,
+                        void* stream) {
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (out_dt != QIFT_F32 && out_dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
+    if (tokens < 0 || n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (set == QIFT_SET_STD) return QIFT_ERR_UNSUPPORTED;
+    if (n_in > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (tokens == 0 || n_out == 0) return QIFT_OK;
+    if (!q_act || !act_scale || !codes || !w_scale || !y) return QIFT_ERR_INVALID_ARG;
+    if (!aligned16(q_act) || !aligned16(codes) || !aligned16(y) || !aligned4(act_scale) || !aligned4(w_scale))
+        return QIFT_ERR_INVALID_ARG;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(qift::launch_linear_gemv(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y,
+                                              out_dt == QIFT_F16, s));
+}
+
+qift_status qift_device_error(void* stream, int32_t* detail) {
+    if (detail) *detail = 0;
+    const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return QIFT_ERR_CUDA;
+    return QIFT_OK;
+}
+
+const char* qift_status_string(qift_status status) {
+    switch (status) {
+        case QIFT_OK: return "QIFT_OK";
+        case QIFT_ERR_INVALID_ARG: return "QIFT_ERR_INVALID_ARG: an argument failed host-side validation";
+        case QIFT_ERR_UNSUPPORTED: return "QIFT_ERR_UNSUPPORTED: valid request this build does not implement";
+        case QIFT_ERR_CUDA: return "QIFT_ERR_CUDA: a CUDA launch or runtime call failed";
+        case QIFT_ERR_TIMEOUT: return "QIFT_ERR_TIMEOUT: a bounded on-chip wait gave up";
+        default: return "QIFT_UNKNOWN_STATUS";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// common.cuh -- small helpers shared by the Qift CUDA kernels (sm_100a only).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libqift is written for sm_100a (B200) only"
+#endif
+
+namespace qift {
+
+constexpr int kSetQift = 0;
+constexpr int kSetPot = 1;
+constexpr int kSetStd = 2;
+
+// Integer level table of a set packed as four signed bytes, byte c = level of code c, so that
+// one byte permute (prmt) turns four 2-bit codes into four int8 weights.
+//   Qift {-3,-1,+1,+3}: bytes FD FF 01 03.   PoT {-4,-1,+1,+4}: bytes FC FF 01 04.
+__host__ __device__ constexpr uint32_t level_lut(int set) {
+    return set == kSetPot ? 0x0401FFFCu : 0x0301FFFDu;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) {
+    return __dp4a((int)a, (int)b, c);
+}
+
+// Decode one packed word (16 codes, code k at bits 2k..2k+1) into 16 int8 weights held in
+// four registers, in the order the activations are permuted to:
+//   d0 = codes {0,2,4,6}, d1 = {8,10,12,14}, d2 = {1,3,5,7}, d3 = {9,11,13,15}.
+// even = w & 0x33333333 holds code 2i in nibble i; odd = (w >> 2) & 0x33333333 holds 2i+1.
+// prmt reads the low 16 bits of its selector as four nibbles, each picking one LUT byte.
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t lut, uint32_t d[4]) {
+    const uint32_t even = w & 0x33333333u;
+    const uint32_t odd = (w >> 2) & 0x33333333u;
+    d[0] = prmt(lut, 0u, even);
+    d[1] = prmt(lut, 0u, even >> 16);
+    d[2] = prmt(lut, 0u, odd);
+    d[3] = prmt(lut, 0u, odd >> 16);
+}
+
+// Permute 16 int8 activations (natural order in four words) into the decode_word order.
+__device__ __forceinline__ void permute_acts(uint4 a, uint32_t p[4]) {
+    p[0] = prmt(a.x, a.y, 0x6420u);   // bytes 0,2 of x and 0,2 of y -> k = 0,2,4,6
+    p[1] = prmt(a.z, a.w, 0x6420u);   // k = 8,10,12,14
+    p[2] = prmt(a.x, a.y, 0x7531u);   // k = 1,3,5,7
+    p[3] = prmt(a.z, a.w, 0x7531u);   // k = 9,11,13,15
+}
+
+__host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
+
+}  // namespace qift

@@ -1,0 +1,25 @@
+// internal.h -- launchers shared between the C ABI (api.cu) and the kernel files.
+// Arguments are validated by the caller; launchers only configure and launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qift {
+
+cudaError_t launch_rotate(const void* x, void* y, bool f16, int64_t rows, int64_t n, int block,
+                          cudaStream_t s);
+
+cudaError_t launch_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int block, int8_t* q,
+                                 float* scales, cudaStream_t s);
+
+cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int set, int grid_points,
+                                    double lo, double hi, uint32_t* codes, float* scales, double* row_mse,
+                                    cudaStream_t s);
+
+// Decode-size linear: HBM-streaming GEMV (CUDA-core dp4a).
+cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                               int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
+                               cudaStream_t s);
+
+}  // namespace qift

@@ -1,0 +1,158 @@
+// linear_gemv.cu -- qift_linear at decode batch sizes: an HBM-streaming W2A4 GEMV.
+//
+// "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+// Inference", Abstract: "sign-and-shift decoded weight application" of the fixed 2-bit levels
+// under rotated W2A4 inference.
+//
+// acc[t][n] = sum_k q[t][k] * L(code[n][k])  (int32),  y = ((float)acc * s_w[n]) * s_a[t].
+//
+// Each warp owns R output rows; lane l streams 16-byte groups of packed codes (64 weights)
+// at word offsets 4l + 128j.  Every code load of the warp's rows is issued before any math so
+// the whole weight tile is in flight at once.  A 32-bit word of 16 codes is decoded to int8
+// with two masks, two shifts and four byte permutes against the set's level table (a Qift or
+// power-of-two level is one table byte; for {+-1,+-4} the byte is the sign-and-shift result),
+// and meets the matching activations with dp4a.  The activations of the lane's words are
+// loaded once per chunk, permuted to the decode order, and reused across the R rows.
+#include "common.cuh"
+#include "internal.h"
+
+namespace qift {
+
+constexpr int kGemvWarps = 4;
+
+template <typename OutT>
+__device__ __forceinline__ void store_out(OutT* p, float v);
+template <>
+__device__ __forceinline__ void store_out<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void store_out<__half>(__half* p, float v) { *p = __float2half_rn(v); }
+
+// TC tokens per CTA row of the grid (blockIdx.y picks the token chunk), R rows per warp,
+// J 128-word slices per K chunk, VEC = codes rows are 16-byte aligned (K % 64 == 0).
+template <int TC, int R, int J, bool VEC, typename OutT>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __restrict__ q,
+                                                               const float* __restrict__ s_a,
+                                                               const uint32_t* __restrict__ codes,
+                                                               const float* __restrict__ s_w, uint32_t lut,
+                                                               int64_t T, int64_t N, int64_t K,
+                                                               OutT* __restrict__ y) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t)blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
+    const int64_t row0 = warp * R;
+    const int64_t t0 = (int64_t)blockIdx.y * TC;
+    const int64_t KW = K / 16;
+    int acc[R][TC];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int t = 0; t < TC; ++t) acc[r][t] = 0;
+
+    for (int64_t base = 0; base < KW; base += 128 * J) {
+        // 1. Issue all code loads for this chunk (R rows x J slices x 4 words).
+        uint4 cw[R][J];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int64_t n = row0 + r;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int64_t wi = base + 4 * lane + 128 * j;
+                uint4 c = make_uint4(0u, 0u, 0u, 0u);
+                if (n < N) {
+                    const uint32_t* p = codes + n * KW + wi;
+                    if (VEC && wi + 4 <= KW) {
+                        c = __ldg(reinterpret_cast<const uint4*>(p));
+                    } else {
+                        if (wi + 0 < KW) c.x = __ldg(p + 0);
+                        if (wi + 1 < KW) c.y = __ldg(p + 1);
+                        if (wi + 2 < KW) c.z = __ldg(p + 2);
+                        if (wi + 3 < KW) c.w = __ldg(p + 3);
+                    }
+                }
+                cw[r][j] = c;
+            }
+        }
+        // 2. Activations of the lane's words, permuted to the decode order.
+        uint32_t pa[TC][J][4][4];
+#pragma unroll
+        for (int t = 0; t < TC; ++t) {
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t wi = base + 4 * lane + 128 * j + u;
+                    uint4 a = make_uint4(0u, 0u, 0u, 0u);
+                    if (t0 + t < T && wi < KW) a = __ldg(reinterpret_cast<const uint4*>(q + (t0 + t) * K + wi * 16));
+                    permute_acts(a, pa[t][j][u]);
+                }
+            }
+        }
+        // 3. Decode and accumulate.
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const uint32_t words[4] = {cw[r][j].x, cw[r][j].y, cw[r][j].z, cw[r][j].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t d[4];
+                    decode_word(words[u], lut, d);
+#pragma unroll
+                    for (int t = 0; t < TC; ++t) {
+                        int a = acc[r][t];
+                        a = dp4a(d[0], pa[t][j][u][0], a);
+                        a = dp4a(d[1], pa[t][j][u][1], a);
+                        a = dp4a(d[2], pa[t][j][u][2], a);
+                        a = dp4a(d[3], pa[t][j][u][3], a);
+                        acc[r][t] = a;
+                    }
+                }
+            }
+        }
+    }
+    // 4. Warp reduction and the fp32 epilogue.
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int t = 0; t < TC; ++t) {
+            const int sum = __reduce_add_sync(0xffffffffu, acc[r][t]);
+            const int64_t n = row0 + r, tt = t0 + t;
+            if (lane == ((r * TC + t) & 31) && n < N && tt < T) {
+                const float v = __fmul_rn(__fmul_rn((float)sum, s_w[n]), s_a[tt]);
+                store_out<OutT>(y + tt * N + n, v);
+            }
+        }
+    }
+}
+
+template <int TC, int R, int J, typename OutT>
+static cudaError_t launch_gemv_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                 uint32_t lut, int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    const int64_t warps = (N + R - 1) / R;
+    const int64_t gx = (warps + kGemvWarps - 1) / kGemvWarps;
+    const int64_t gy = (T + TC - 1) / TC;
+    if (gx > 0x7fffffff || gy > 65535) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)gx, (unsigned)gy);
+    if ((K / 16) % 4 == 0)
+        gemv_kernel<TC, R, J, true, OutT><<<grid, kGemvWarps * 32, 0, s>>>(q, s_a, codes, s_w, lut, T, N, K, y);
+    else
+        gemv_kernel<TC, R, J, false, OutT><<<grid, kGemvWarps * 32, 0, s>>>(q, s_a, codes, s_w, lut, T, N, K, y);
+    return cudaGetLastError();
+}
+
+template <typename OutT>
+static cudaError_t dispatch_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                 uint32_t lut, int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    if (T == 1) return launch_gemv_t<1, 4, 2, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
+    if (T == 2) return launch_gemv_t<2, 4, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
+    return launch_gemv_t<4, 2, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
+}
+
+cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                               int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (f16) return dispatch_gemv<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return dispatch_gemv<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
+
+}  // namespace qift

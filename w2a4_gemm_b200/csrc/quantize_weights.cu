@@ -1,0 +1,180 @@
+// quantize_weights.cu -- qift_quantize_weights: per-output-channel MSE scale search, nearest-
+// level encoding and 2-bit packing for the Qift {+-1,+-3}, power-of-two {+-1,+-4} and
+// standard {-2,-1,0,+1} level sets.
+//
+// "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+// Inference", Abstract: a fixed two-bit code-to-level mapping with the standard per-channel
+// scale (no zero point, no group grid).
+//
+// One CTA owns one output row.  The row is staged in shared memory; thread g evaluates
+// candidate scale s_g by walking the row in index order and accumulating the fp32 squared
+// error into fp64 -- the fixed order makes the argmin reproducible bit for bit.  This pass is
+// ALU-bound (G candidates x K elements per row), not HBM-bound.
+//
+// Level thresholds are compared in fp32 against products rounded DOWN: for a float x and a
+// real threshold tau = c*s, x > tau exactly when x > RD(c*s), because no float lies strictly
+// between RD(c*s) and RU(c*s).  That decides every weight exactly as an exact comparison would.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qift {
+
+constexpr int kQwThreads = 128;
+
+template <int SET>
+struct Encoder {
+    float s, thr1, thr2, l_in, l_out;
+    __device__ __forceinline__ explicit Encoder(float s_) : s(s_) {
+        if constexpr (SET == kSetQift) {        // levels +-0.5 s, +-1.5 s; midpoint s
+            thr1 = s;
+            l_in = __fmul_rn(0.5f, s);
+            l_out = __fmul_rn(1.5f, s);
+        } else if constexpr (SET == kSetPot) {  // levels +-s, +-4 s; midpoint 2.5 s
+            thr1 = __fmul_rd(2.5f, s);
+            l_in = s;
+            l_out = __fmul_rn(4.0f, s);
+        } else {                                // levels -2s, -s, 0, s; midpoints -1.5s, -0.5s, 0.5s
+            thr1 = __fmul_rd(1.5f, s);
+            thr2 = __fmul_rd(0.5f, s);
+        }
+    }
+    // Code 0..3 (monotone in level).  Ties go to the smaller magnitude; w >= 0 is positive.
+    __device__ __forceinline__ uint32_t code(float w) const {
+        if constexpr (SET == kSetStd) {
+            const float nw = -w;
+            if (nw > thr1) return 0u;   // w < -1.5 s
+            if (nw > thr2) return 1u;   // w < -0.5 s
+            if (w > thr2) return 3u;    // w > +0.5 s
+            return 2u;
+        } else {
+            const bool outer = fabsf(w) > thr1;
+            return w >= 0.0f ? (outer ? 3u : 2u) : (outer ? 0u : 1u);
+        }
+    }
+    // Squared reconstruction error of w, in fp32, for its code.
+    __device__ __forceinline__ float sq_err(float w) const {
+        float e;
+        if constexpr (SET == kSetStd) {
+            const float l = __fmul_rn((float)((int)code(w) - 2), s);
+            e = __fsub_rn(w, l);
+        } else {
+            const float a = fabsf(w);
+            e = __fsub_rn(a, a > thr1 ? l_out : l_in);
+        }
+        return __fmul_rn(e, e);
+    }
+};
+
+template <int SET>
+__global__ void __launch_bounds__(kQwThreads) quant_weights_kernel(const float* __restrict__ w, int64_t K, int G,
+                                                                   double lo, double hi,
+                                                                   uint32_t* __restrict__ codes,
+                                                                   float* __restrict__ scales,
+                                                                   double* __restrict__ row_mse) {
+    extern __shared__ __align__(16) float ws[];  // the row, K floats
+    __shared__ float cand[256];
+    __shared__ double mse[256];
+    __shared__ float red[kQwThreads / 32];
+    __shared__ int best_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const float* wr = w + row * K;
+
+    // Stage the row and find max |w|.
+    float m = 0.0f;
+    for (int64_t i = (int64_t)tid * 4; i < K; i += kQwThreads * 4) {
+        const float4 v = *reinterpret_cast<const float4*>(wr + i);
+        *reinterpret_cast<float4*>(ws + i) = v;
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+
+    // Candidate scales, binary64 in the order lo + ((hi - lo) * k) / (G - 1), then * m / L.
+    const double lambda = SET == kSetQift ? 1.5 : (SET == kSetPot ? 4.0 : 2.0);
+    for (int g = tid; g < G; g += kQwThreads) {
+        const double f = __dadd_rn(lo, __ddiv_rn(__dmul_rn(__dsub_rn(hi, lo), (double)g), (double)(G - 1)));
+        cand[g] = __double2float_rn(__ddiv_rn(__dmul_rn(f, (double)m), lambda));
+    }
+    __syncthreads();
+
+    // MSE of every candidate: sequential over the row, fp32 squared error widened to fp64.
+    for (int g = tid; g < G; g += kQwThreads) {
+        const Encoder<SET> enc(cand[g]);
+        double acc = 0.0;
+        const float4* w4 = reinterpret_cast<const float4*>(ws);
+        for (int64_t i = 0; i < K / 4; ++i) {
+            const float4 v = w4[i];
+            acc = __dadd_rn(acc, (double)enc.sq_err(v.x));
+            acc = __dadd_rn(acc, (double)enc.sq_err(v.y));
+            acc = __dadd_rn(acc, (double)enc.sq_err(v.z));
+            acc = __dadd_rn(acc, (double)enc.sq_err(v.w));
+        }
+        mse[g] = acc;
+    }
+    __syncthreads();
+
+    // Argmin, first index on ties.
+    if (tid == 0) {
+        int b = 0;
+        double bv = mse[0];
+        for (int g = 1; g < G; ++g)
+            if (mse[g] < bv) { bv = mse[g]; b = g; }
+        best_s = b;
+    }
+    __syncthreads();
+    const int b = best_s;
+    const float s = cand[b];
+    const Encoder<SET> enc(s);
+
+    // Encode and pack: word j holds the codes of inputs 16j .. 16j+15, 2 bits each.
+    uint32_t* crow = codes + row * (K / 16);
+    for (int64_t j = tid; j < K / 16; j += kQwThreads) {
+        const float4* w4 = reinterpret_cast<const float4*>(ws + j * 16);
+        uint32_t word = 0;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+            const float4 v = w4[v4];
+            word |= enc.code(v.x) << (8 * v4);
+            word |= enc.code(v.y) << (8 * v4 + 2);
+            word |= enc.code(v.z) << (8 * v4 + 4);
+            word |= enc.code(v.w) << (8 * v4 + 6);
+        }
+        crow[j] = word;
+    }
+    if (tid == 0) {
+        scales[row] = SET == kSetQift ? __fmul_rn(s, 0.5f) : s;
+        if (row_mse) row_mse[row] = __ddiv_rn(mse[b], (double)K);
+    }
+}
+
+template <int SET>
+static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
+                             uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
+    const size_t smem = (size_t)n_in * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(quant_weights_kernel<SET>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    quant_weights_kernel<SET><<<(unsigned)n_out, kQwThreads, smem, s>>>(w, n_in, G, lo, hi, codes, scales, row_mse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int set, int G, double lo,
+                                    double hi, uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
+    if (n_out == 0) return cudaSuccess;
+    switch (set) {
+        case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
+        case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
+        case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace qift
