@@ -189,3 +189,16 @@ def test_single_linear_256x512_end_to_end():
     assert np.array_equal(host(gq), ref["q"])
     tol_check(host(gy), ref["y"], 1e-5)
     assert np.array_equal(host(gy), ref["y"])
+
+
+# ------------------------------------------------------------- tensor-core GEMM (prefill)
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("T,N,K", [(17, 256, 64), (128, 256, 128), (129, 257, 192), (300, 600, 4096),
+                                    (256, 40, 640), (2048, 512, 11008), (64, 1000, 4160)])
+def test_linear_gemm_parity(name, T, N, K):
+    for out_dtype in (torch.float16, torch.float32):
+        got, ref = _linear_case(name, T, N, K, T + 7 * N + K, out_dtype)
+        tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
+        assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
+                              ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32))
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)

@@ -79,15 +79,21 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
     if (!aligned16(q_act) || !aligned16(codes) || !aligned16(y) || !aligned4(act_scale) || !aligned4(w_scale))
         return QIFT_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return from_cuda(qift::launch_linear_gemv(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y,
-                                              out_dt == QIFT_F16, s));
+    const bool f16 = out_dt == QIFT_F16;
+    if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
+        return from_cuda(qift::launch_linear_gemm(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y,
+                                                  f16, s));
+    return from_cuda(
+        qift::launch_linear_gemv(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y, f16, s));
 }
 
 qift_status qift_device_error(void* stream, int32_t* detail) {
     if (detail) *detail = 0;
-    const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return QIFT_ERR_CUDA;
-    return QIFT_OK;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QIFT_ERR_CUDA;
+    int word = 0;
+    if (qift::read_and_clear_device_error(&word) != cudaSuccess) return QIFT_ERR_CUDA;
+    if (detail) *detail = word;
+    return word ? QIFT_ERR_TIMEOUT : QIFT_OK;
 }
 
 const char* qift_status_string(qift_status status) {

@@ -54,6 +54,33 @@ __device__ __forceinline__ void permute_acts(uint4 a, uint32_t p[4]) {
     p[3] = prmt(a.z, a.w, 0x7531u);   // k = 9,11,13,15
 }
 
+// Decode one packed word into 16 int8 weights in natural input order: d[j] holds the weights
+// of inputs 4j .. 4j+3.  Each byte of codes (four 2-bit fields) is spread to four nibbles --
+// a byte permute places bytes 0/1 (or 2/3) of w 16 bits apart, then two shift-or-mask steps
+// move every 2-bit field into its own nibble -- and one byte permute per four codes reads
+// the level table.
+__device__ __forceinline__ uint32_t spread_codes_to_nibbles(uint32_t two_bytes_16_apart) {
+    uint32_t x = two_bytes_16_apart;
+    x = (x | (x << 4)) & 0x0F0F0F0Fu;
+    x = (x | (x << 2)) & 0x33333333u;
+    return x;
+}
+
+__device__ __forceinline__ void decode_word_natural(uint32_t w, uint32_t lut, uint32_t d[4]) {
+    const uint32_t lo = spread_codes_to_nibbles(prmt(w, 0u, 0x4140u));   // codes 0..7
+    const uint32_t hi = spread_codes_to_nibbles(prmt(w, 0u, 0x4342u));   // codes 8..15
+    d[0] = prmt(lut, 0u, lo);
+    d[1] = prmt(lut, 0u, lo >> 16);
+    d[2] = prmt(lut, 0u, hi);
+    d[3] = prmt(lut, 0u, hi >> 16);
+}
+
+// Programmatic dependent launch.  wait: block until the kernels this launch depends on have
+// completed and their writes are visible (a no-op without a programmatic dependency).
+// launch_dependents: allow the next kernel on the stream to start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
 
 }  // namespace qift

@@ -22,4 +22,16 @@ cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t
                                int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                cudaStream_t s);
 
+// Prefill-size linear: tcgen05 int8 tensor-core GEMM with in-register code decode.
+bool linear_gemm_supported(int64_t tokens, int64_t n_out, int64_t n_in);
+cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                               int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
+                               cudaStream_t s);
+
+// Synchronous read-and-clear of the device error word set by bounded on-chip waits.
+cudaError_t read_and_clear_device_error(int* word);
+
+// Token count from which qift_linear uses the tensor-core GEMM instead of the GEMV.
+constexpr int64_t kGemmMinTokens = 17;
+
 }  // namespace qift

@@ -1,0 +1,333 @@
+// linear_gemm_tc.cu -- qift_linear at prefill batch sizes: a fused W2A4 GEMM on the sm_100a
+// tensor cores (tcgen05, int8 x int8 -> int32 in tensor memory).
+//
+// "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+// Inference", Abstract: 2-bit weights with fixed levels ({+-1,+-3} or {+-1,+-4} times the
+// per-channel scale) applied to 4-bit activations.
+//
+//   y[t][n] = ((float)acc[t][n] * s_w[n]) * s_a[t],  acc = sum_k q[t][k] * L(code[n][k]).
+//
+// One CTA computes a 128-token x 256-output tile, walking K in 128-byte blocks through a
+// 3-stage shared-memory ring:
+//   warp 0      TMA producer: the int8 activation tile (128 x 128 B, 128-byte swizzle) and the
+//               packed code tile (256 rows x 8 words) land on one mbarrier per stage;
+//   warps 2..5  decoders: expand 2-bit codes to int8 weights in registers (byte permutes
+//               against the level table) and write them in the tensor core's 128-byte
+//               swizzled K-major layout; then, after the last block, the epilogue:
+//               tcgen05.ld of the int32 accumulators, the fp32 scale product, stores;
+//   warp 1      allocates 256 TMEM columns and one elected thread issues tcgen05.mma
+//               (kind::i8, M=128, N=256, K=32 per instruction, 4 per block), committing each
+//               stage back to the producer.
+// Every mbarrier wait is bounded: a wait that runs out of time sets a shared abort flag and
+// the device error word, every role drains what it started, TMEM is freed and the CTA exits.
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tc.cuh"
+
+namespace qift {
+
+__device__ int g_qift_error = 0;  // QIFT_ERR_TIMEOUT-style bits, read by qift_device_error()
+
+namespace gemm {
+
+constexpr int BM = 128;          // tokens per tile (MMA M, TMEM lanes)
+constexpr int BN = 256;          // output features per tile (MMA N, TMEM columns)
+constexpr int BK = 128;          // K bytes per stage (one 128-byte swizzle row)
+constexpr int STAGES = 3;
+constexpr int kThreads = 192;    // 6 warps
+constexpr int A_BYTES = BM * BK;             // 16 KB
+constexpr int B_BYTES = BN * BK;             // 32 KB
+constexpr int C_BYTES = BN * (BK / 16) * 4;  // 8 KB of packed codes
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + C_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz before a wait gives up
+
+struct Smem {
+    uint8_t* a;
+    uint8_t* b;
+    uint8_t* c;
+    uint64_t* full;
+    uint64_t* decoded;
+    uint64_t* empty;
+    uint64_t* accum;
+    uint32_t* tmem_base;
+    int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    Smem s;
+    s.a = base;
+    s.b = s.a + STAGES * A_BYTES;
+    s.c = s.b + STAGES * B_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.c + STAGES * C_BYTES);
+    s.full = bars;
+    s.decoded = bars + STAGES;
+    s.empty = bars + 2 * STAGES;
+    s.accum = bars + 3 * STAGES;
+    s.tmem_base = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+    s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
+    return s;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* abort) {
+    if (tc::mbar_wait_bounded(bar, parity, abort, kWaitCycles)) return true;
+    if (!*reinterpret_cast<volatile int*>(abort)) {
+        atomicOr(&g_qift_error, 1);
+        *reinterpret_cast<volatile int*>(abort) = 1;
+    }
+    return false;
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_row16(OutT* y, int64_t row, int64_t n0, int64_t N, const float* v);
+
+template <>
+__device__ __forceinline__ void store_row16<__half>(__half* y, int64_t row, int64_t n0, int64_t N, const float* v) {
+    __half* p = y + row * N + n0;
+    if ((N & 7) == 0 && n0 + 16 <= N) {
+        uint4 t0, t1;
+        __half2* h0 = reinterpret_cast<__half2*>(&t0);
+        __half2* h1 = reinterpret_cast<__half2*>(&t1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h0[j] = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+            h1[j] = __floats2half2_rn(v[8 + 2 * j], v[8 + 2 * j + 1]);
+        }
+        reinterpret_cast<uint4*>(p)[0] = t0;
+        reinterpret_cast<uint4*>(p)[1] = t1;
+    } else {
+        for (int j = 0; j < 16; ++j)
+            if (n0 + j < N) p[j] = __float2half_rn(v[j]);
+    }
+}
+
+template <>
+__device__ __forceinline__ void store_row16<float>(float* y, int64_t row, int64_t n0, int64_t N, const float* v) {
+    float* p = y + row * N + n0;
+    if ((N & 3) == 0 && n0 + 16 <= N) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4*>(p)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+        for (int j = 0; j < 16; ++j)
+            if (n0 + j < N) p[j] = v[j];
+    }
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    w2a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_c,
+                     const float* __restrict__ s_a, const float* __restrict__ s_w, uint32_t lut, int T, int N,
+                     int K, OutT* __restrict__ y) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;
+    const int m0 = blockIdx.y * BM;
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.decoded[s], 128);
+            tc::mbar_init(&sm.empty[s], 1);
+        }
+        tc::mbar_init(sm.accum, 1);
+        *sm.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&tmap_a);
+        tc::prefetch_tensormap(&tmap_c);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_d = *sm.tmem_base;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t round = kb / STAGES;
+                if (!wait_or_abort(&sm.empty[s], (round & 1) ^ 1, sm.abort)) break;
+                tc::mbar_arrive_expect_tx(&sm.full[s], A_BYTES + C_BYTES);
+                tc::tma_load_2d(sm.a + s * A_BYTES, &tmap_a, &sm.full[s], kb * BK, m0);
+                tc::tma_load_2d(sm.c + s * C_BYTES, &tmap_c, &sm.full[s], kb * (BK / 16), n0);
+                ++issued;
+            }
+            if (*reinterpret_cast<volatile int*>(sm.abort)) {
+                // Drain: let every copy this thread started land before the CTA exits.
+                int zero = 0;
+                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
+                    tc::mbar_wait_bounded(&sm.full[kb % STAGES], (kb / STAGES) & 1, &zero, kWaitCycles);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_i8(BM, BN);
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                const uint32_t parity = (kb / STAGES) & 1;
+                if (!wait_or_abort(&sm.full[s], parity, sm.abort)) break;
+                if (!wait_or_abort(&sm.decoded[s], parity, sm.abort)) break;
+                tc::tc_fence_after();
+                const uint32_t a_addr = tc::smem_u32(sm.a + s * A_BYTES);
+                const uint32_t b_addr = tc::smem_u32(sm.b + s * B_BYTES);
+#pragma unroll
+                for (int k = 0; k < BK / 32; ++k) {
+                    tc::mma_i8_ss(tmem_d, tc::smem_desc_sw128(a_addr + 32 * k), tc::smem_desc_sw128(b_addr + 32 * k),
+                                  idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(&sm.empty[s]);
+            }
+            tc::mma_commit(sm.accum);  // also issued after an abort, so TMEM is idle before it is freed
+        }
+    } else {
+        // ---------------------------------------------------------------- decoders
+        const int d = threadIdx.x - 64;  // 0..127: rows d and d + 128 of the weight tile
+        for (int kb = 0; kb < num_kb; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t parity = (kb / STAGES) & 1;
+            if (!wait_or_abort(&sm.full[s], parity, sm.abort)) break;
+            const uint8_t* ctile = sm.c + s * C_BYTES;
+            uint8_t* btile = sm.b + s * B_BYTES;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = d + 128 * h;
+                const uint4 w0 = *reinterpret_cast<const uint4*>(ctile + r * 32);
+                const uint4 w1 = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16);
+                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint8_t* brow = btile + r * BK;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t v[4];
+                    decode_word_natural(words[c], lut, v);
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&sm.decoded[s]);
+        }
+        // ---------------------------------------------------------------- epilogue
+        bool ok = wait_or_abort(sm.accum, 0, sm.abort) && !*reinterpret_cast<volatile int*>(sm.abort);
+        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective: decide per warp
+        if (ok) {
+            tc::tc_fence_after();
+            const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
+            const int row = m0 + quarter * 32 + lane;  // token
+            const float sa = row < T ? s_a[row] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 16; ++cc) {
+                uint32_t acc[16];
+                tc::tmem_ld_32x32b_x16(tmem_d + ((uint32_t)(quarter * 32) << 16) + cc * 16, acc);
+                tc::tmem_ld_wait();
+                const int nb = n0 + cc * 16;
+                if (row < T && nb < N) {
+                    float v[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float sw = (nb + j < N) ? s_w[nb + j] : 0.0f;
+                        v[j] = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sa);
+                    }
+                    store_row16<OutT>(y, row, nb, N, v);
+                }
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        // Every MMA this CTA issued has been committed to sm.accum; make sure they are done.
+        __syncwarp();
+        int zero = 0;
+        tc::mbar_wait_bounded(sm.accum, 0, &zero, kWaitCycles);
+        __syncwarp();
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_d, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+template <typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    auto encode = get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap ma, mc;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {BK, BM};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16) * 4};
+        const cuuint32_t box[2] = {BK / 16, BN};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(w2a4_gemm_kernel<OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((T + BM - 1) / BM));
+    w2a4_gemm_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(ma, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y);
+    return cudaGetLastError();
+}
+
+}  // namespace gemm
+
+bool linear_gemm_supported(int64_t T, int64_t N, int64_t K) {
+    // TMA needs 16-byte row strides for the code matrix (K % 64) and the grid fits.
+    return K % 64 == 0 && T <= (int64_t)65535 * gemm::BM && N <= (int64_t)0x7fffffff;
+}
+
+cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                               int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (f16) return gemm::launch_t<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return gemm::launch_t<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
+
+cudaError_t read_and_clear_device_error(int* word) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_qift_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    if (v != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_qift_error, &zero, sizeof(int));
+    }
+    *word = v;
+    return e;
+}
+
+}  // namespace qift

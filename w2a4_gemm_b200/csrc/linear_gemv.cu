@@ -47,9 +47,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
 #pragma unroll
         for (int t = 0; t < TC; ++t) acc[r][t] = 0;
 
-    for (int64_t base = 0; base < KW; base += 128 * J) {
-        // 1. Issue all code loads for this chunk (R rows x J slices x 4 words).
-        uint4 cw[R][J];
+    // Codes of one K chunk (R rows x J slices x 4 words) straight into registers.
+    uint4 cw[R][J];
+    auto load_codes = [&](int64_t base) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int64_t n = row0 + r;
@@ -71,6 +71,16 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
                 cw[r][j] = c;
             }
         }
+    };
+    // 1. The first chunk of codes is requested before waiting for the previous kernel on the
+    //    stream (programmatic dependent launch): the weight stream overlaps its tail.  Only
+    //    codes are read before the wait; activations, scales and y come after it.
+    load_codes(0);
+    griddep_launch_dependents();
+    griddep_wait();
+
+    for (int64_t base = 0; base < KW; base += 128 * J) {
+        if (base > 0) load_codes(base);
         // 2. Activations of the lane's words, permuted to the decode order.
         uint32_t pa[TC][J][4][4];
 #pragma unroll
@@ -131,12 +141,18 @@ static cudaError_t launch_gemv_t(const int8_t* q, const float* s_a, const uint32
     const int64_t gx = (warps + kGemvWarps - 1) / kGemvWarps;
     const int64_t gy = (T + TC - 1) / TC;
     if (gx > 0x7fffffff || gy > 65535) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)gx, (unsigned)gy);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)gx, (unsigned)gy);
+    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if ((K / 16) % 4 == 0)
-        gemv_kernel<TC, R, J, true, OutT><<<grid, kGemvWarps * 32, 0, s>>>(q, s_a, codes, s_w, lut, T, N, K, y);
-    else
-        gemv_kernel<TC, R, J, false, OutT><<<grid, kGemvWarps * 32, 0, s>>>(q, s_a, codes, s_w, lut, T, N, K, y);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, gemv_kernel<TC, R, J, true, OutT>, q, s_a, codes, s_w, lut, T, N, K, y);
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<TC, R, J, false, OutT>, q, s_a, codes, s_w, lut, T, N, K, y);
 }
 
 template <typename OutT>

@@ -44,6 +44,10 @@ __global__ void __launch_bounds__(kActThreads) quant_acts_kernel(const __half* _
     const int64_t token = blockIdx.x;
     const __half* xt = x + token * K;
     float amax = 0.0f;
+    // Launched as a programmatic dependent: wait for the previous kernel on the stream before
+    // touching memory, then let the next one (the linear) start its weight stream early.
+    griddep_wait();
+    griddep_launch_dependents();
 
     if constexpr (LOGB == 0) {
         for (int64_t i = (int64_t)tid * 8; i < K; i += kActThreads * 8) {
@@ -140,8 +144,17 @@ static cudaError_t launch_qa(const __half* x, int64_t tokens, int64_t K, int8_t*
                                              (int)smem);
         if (e != cudaSuccess) return e;
     }
-    quant_acts_kernel<LOGB><<<(unsigned)tokens, kActThreads, smem, s>>>(x, K, q, scales, c);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tokens);
+    cfg.blockDim = dim3(kActThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quant_acts_kernel<LOGB>, x, K, q, scales, c);
 }
 
 cudaError_t launch_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int block, int8_t* q, float* scales,
