@@ -160,15 +160,49 @@ class OursState:
         return 2 * len(self.layers)
 
 
-def time_region(torch, fn, iters):
+def max_over_ranks(value: float, world: int) -> float:
+    """The largest of every rank's value (one all-reduce); the value itself on one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def capture(torch, fn, iters, offset=0):
+    """A CUDA graph of fn(offset) .. fn(offset + iters - 1): the launches go through the C ABI
+    onto the capturing stream, so replaying the graph replays exactly those kernels."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(iters):
+            fn(offset + i)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, g):
+    """Seconds of one replay, CUDA events on the replaying stream, synchronised both sides."""
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     s.record()
-    for i in range(iters):
-        fn(i)
+    g.replay()
     e.record()
     torch.cuda.synchronize()
-    return s.elapsed_time(e) / 1e3  # seconds
+    return s.elapsed_time(e) / 1e3
+
+
+def time_region(torch, fn, iters):
+    """Seconds for fn(0..iters-1) replayed as one CUDA graph (captured, uploaded, then timed)."""
+    g = capture(torch, fn, iters)
+    g.replay()
+    torch.cuda.synchronize()
+    return time_graph(torch, g)
 
 
 def run_ours(args, rank, world):
@@ -195,18 +229,18 @@ def run_ours(args, rank, world):
         st.step(i)
     torch.cuda.synchronize()
 
-    dist = None
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+    g_steps = capture(torch, st.step, args.steps, offset=args.warmup)
+    g_steps.replay()  # upload and warm the graph itself (not timed)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        secs = time_region(torch, st.step, args.steps)
-        if world > 1:
-            t = torch.tensor([secs], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            secs = float(t.item())
+        secs = max_over_ranks(time_graph(torch, g_steps), world)
     clocks = clk.summary()
+    del g_steps
 
     # Per-kernel live timing over the same cycled inputs (one kernel type per loop).
     L0 = st.layers[0]
@@ -269,11 +303,7 @@ def run_ours(args, rank, world):
 
     for i in range(args.warmup):
         e2e_step(i)
-    e2e_secs = time_region(torch, e2e_step, args.steps)
-    if world > 1:
-        t = torch.tensor([e2e_secs], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_secs = float(t.item())
+    e2e_secs = max_over_ranks(time_region(torch, e2e_step, args.steps), world)
     h2d = sum(x.numel() * x.element_size() for x in hx)
     d2h = sum(y.numel() * y.element_size() for y in hy)
     e2e_val = world * (step_bytes if decode else step_ops) * args.steps / e2e_secs / (1e9 if decode else 1e12)

@@ -93,6 +93,8 @@ qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_i
  *   scales : fp32 [tokens] out, s_a = m / 7 with m = max |x'| of the token.
  * x' is the rotated token rounded once to fp16; q = clamp(rint(x' * (7/m)), -7, 7) with
  * round-half-even and one fp32 division for 7/m; an all-zero token gives q = 0, s_a = 0.
+ * Launched as a programmatic dependent: it waits for the previous kernel on `stream` before
+ * touching memory, then lets the following qift_linear start its weight stream early.
  */
 qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int32_t block, int8_t* q,
                                float* scales, void* stream);
@@ -107,8 +109,14 @@ qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int3
  *   y         : [tokens][n_out] out, out_dt QIFT_F32 or QIFT_F16 (round to nearest even).
  *   n_in      : multiple of 16, at most 32768 (so |acc| <= 7*4*n_in < 2^24 and (float)acc is
  *               exact).  tokens == 0 or n_out == 0 is a no-op.
- * Decode-size batches (few tokens) run as an HBM-streaming GEMV; larger batches as an int8
- * tensor-core GEMM.  Both give bit-identical results.
+ * Decode-size batches (tokens <= 16) run as an HBM-streaming GEMV; larger batches as an int8
+ * tensor-core GEMM (n_in % 64 == 0; otherwise the GEMV).  Both give bit-identical results.
+ * Overlap: the decode GEMV is launched as a programmatic dependent of the previous kernel on
+ * `stream` and may start reading `codes` -- and only `codes` -- before that kernel has
+ * finished; q_act, act_scale, w_scale and y are touched only after it has completed.  So the
+ * kernel launched immediately before qift_linear on the same stream must not write `codes`
+ * (the usual order qift_quantize_weights -> qift_quantize_acts -> qift_linear satisfies
+ * this: qift_quantize_acts waits for its predecessor before it lets qift_linear start).
  */
 qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint32_t* codes,
                         const float* w_scale, qift_levelset set, int64_t tokens, int64_t n_out,

@@ -1,0 +1,32 @@
+/*
+ * qift_debug.h -- test hooks of libqift.so.  Not part of the computing interface: they exist
+ * so a test can drive the bounded-wait failure path of the tensor-core GEMM on a real GPU
+ * without faulting, trapping or hanging it.
+ */
+#ifndef QIFT_DEBUG_H_
+#define QIFT_DEBUG_H_
+
+#include <stdint.h>
+
+#include "qift.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Give every on-chip wait of later tensor-core GEMM launches at most `cycles` SM clock cycles
+ * before it gives up (default about 4e9, some two seconds).  cycles <= 0 restores the default.
+ * Process-wide; not thread-safe against concurrent qift_linear calls. */
+qift_status qift_debug_set_wait_limit(int64_t cycles);
+
+/* Make the next tensor-core GEMM launch (qift_linear with tokens >= 17) wait, in its MMA-issuing
+ * thread, on a barrier that nothing ever arrives on.  That wait runs out after the wait limit,
+ * the kernel abandons its tile, drains its copies, frees tensor memory and exits; the output is
+ * left unspecified and qift_device_error() then reports QIFT_ERR_TIMEOUT.  One-shot. */
+qift_status qift_debug_stall_next_gemm(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QIFT_DEBUG_H_ */

@@ -1,0 +1,57 @@
+"""Host-side pieces of bench.py: algorithmic byte counts and the max-over-ranks timing
+reduction, the latter with two gloo ranks on the CPU (the N-GPU replica path)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_linear_bytes_q_proj_decode():
+    # codes + w scales + int8 activations + act scale + fp16 output for 4096x4096, one token
+    assert bench.linear_bytes(1, 4096, 4096, 2) == 4096 * 4096 // 4 + 4 * 4096 + 4096 + 4 + 2 * 4096
+    assert bench.acts_bytes(1, 4096) == 3 * 4096 + 4
+
+
+def test_peaks_reads_measured_file_or_fallback():
+    p = bench.peaks()
+    assert p["hbm_gbs"] > 1000 and p["int8_tops"] > 1000
+    assert p["source"] in ("measured", "fallback")
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out[rank] = bench.max_over_ranks(1.5 + rank, world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == out[1] == 2.5
+
+
+def test_max_over_ranks_single_process_is_identity():
+    assert bench.max_over_ranks(3.25, 1) == 3.25

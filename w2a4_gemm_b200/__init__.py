@@ -47,10 +47,12 @@ def lib() -> C.CDLL:
         L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
         L.qift_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, i32, vp]
         L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
+        L.qift_debug_set_wait_limit.argtypes = [i64]
+        L.qift_debug_stall_next_gemm.argtypes = []
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear",
-                     "qift_device_error"):
+                     "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -157,3 +159,13 @@ def qift_device_error(stream=None) -> tuple[int, int]:
     detail = C.c_int32(0)
     st = lib().qift_device_error(_stream(stream), C.byref(detail))
     return st, detail.value
+
+
+def qift_debug_set_wait_limit(cycles: int) -> None:
+    """Test hook: SM-cycle limit of every on-chip wait in later tensor-core GEMMs (<= 0: default)."""
+    _check(lib().qift_debug_set_wait_limit(int(cycles)), "qift_debug_set_wait_limit")
+
+
+def qift_debug_stall_next_gemm() -> None:
+    """Test hook: the next tensor-core GEMM waits on a barrier nothing arrives on and times out."""
+    _check(lib().qift_debug_stall_next_gemm(), "qift_debug_stall_next_gemm")

@@ -3,7 +3,11 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "../../include/qift.h"
+#include "../../include/qift_debug.h"
 #include "internal.h"
 
 namespace {
@@ -20,6 +24,25 @@ qift_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QIFT_OK : QIFT_
 bool valid_block(int64_t b) { return is_pow2(b) && b >= 2 && b <= 4096; }
 
 }  // namespace
+
+namespace qift {
+
+cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes) {
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, size_t> granted;  // (kernel, device) -> bytes allowed
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t key = (reinterpret_cast<uintptr_t>(kernel) << 8) ^ (uint64_t)(dev & 0xff);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = granted.find(key);
+    if (it != granted.end() && it->second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) granted[key] = bytes;
+    return e;
+}
+
+}  // namespace qift
 
 extern "C" {
 
@@ -94,6 +117,16 @@ qift_status qift_device_error(void* stream, int32_t* detail) {
     if (qift::read_and_clear_device_error(&word) != cudaSuccess) return QIFT_ERR_CUDA;
     if (detail) *detail = word;
     return word ? QIFT_ERR_TIMEOUT : QIFT_OK;
+}
+
+qift_status qift_debug_set_wait_limit(int64_t cycles) {
+    qift::debug_set_gemm_wait_limit((long long)cycles);
+    return QIFT_OK;
+}
+
+qift_status qift_debug_stall_next_gemm(void) {
+    qift::debug_stall_next_gemm();
+    return QIFT_OK;
 }
 
 const char* qift_status_string(qift_status status) {

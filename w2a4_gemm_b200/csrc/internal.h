@@ -3,9 +3,20 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 namespace qift {
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device), so launches --
+// including ones captured into CUDA graphs -- do not repeat the attribute call.
+cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes);
+
+template <typename Kernel>
+inline cudaError_t ensure_smem(Kernel kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return ensure_smem_ptr(reinterpret_cast<const void*>(kernel), bytes);
+}
 
 cudaError_t launch_rotate(const void* x, void* y, bool f16, int64_t rows, int64_t n, int block,
                           cudaStream_t s);
@@ -27,6 +38,10 @@ bool linear_gemm_supported(int64_t tokens, int64_t n_out, int64_t n_in);
 cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                cudaStream_t s);
+
+// Test hooks behind qift_debug.h.
+void debug_set_gemm_wait_limit(long long cycles);
+void debug_stall_next_gemm();
 
 // Synchronous read-and-clear of the device error word set by bounded on-chip waits.
 cudaError_t read_and_clear_device_error(int* word);

@@ -43,6 +43,11 @@ constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + C_BYTES) + 1024 /*align
 constexpr uint32_t TMEM_COLS = 256;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz before a wait gives up
 
+// Test hooks (qift_debug.h): a shorter wait limit, and a one-shot stall that makes the MMA
+// thread wait on a barrier nothing arrives on, so the timeout path runs without any fault.
+static long long g_wait_limit = kWaitCycles;
+static bool g_stall_next = false;
+
 struct Smem {
     uint8_t* a;
     uint8_t* b;
@@ -51,6 +56,7 @@ struct Smem {
     uint64_t* decoded;
     uint64_t* empty;
     uint64_t* accum;
+    uint64_t* never;
     uint32_t* tmem_base;
     int* abort;
 };
@@ -66,13 +72,14 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.decoded = bars + STAGES;
     s.empty = bars + 2 * STAGES;
     s.accum = bars + 3 * STAGES;
-    s.tmem_base = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+    s.never = bars + 3 * STAGES + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 2);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     return s;
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* abort) {
-    if (tc::mbar_wait_bounded(bar, parity, abort, kWaitCycles)) return true;
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int* abort, long long limit) {
+    if (tc::mbar_wait_bounded(bar, parity, abort, limit)) return true;
     if (!*reinterpret_cast<volatile int*>(abort)) {
         atomicOr(&g_qift_error, 1);
         *reinterpret_cast<volatile int*>(abort) = 1;
@@ -120,7 +127,7 @@ template <typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     w2a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_c,
                      const float* __restrict__ s_a, const float* __restrict__ s_w, uint32_t lut, int T, int N,
-                     int K, OutT* __restrict__ y) {
+                     int K, OutT* __restrict__ y, long long wait_limit, int stall) {
     extern __shared__ uint8_t smem_raw[];
     const Smem sm = carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -135,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&sm.empty[s], 1);
         }
         tc::mbar_init(sm.accum, 1);
+        tc::mbar_init(sm.never, 1);
         *sm.abort = 0;
         tc::fence_mbar_init();
         tc::prefetch_tensormap(&tmap_a);
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < num_kb; ++kb) {
                 const int s = kb % STAGES;
                 const uint32_t round = kb / STAGES;
-                if (!wait_or_abort(&sm.empty[s], (round & 1) ^ 1, sm.abort)) break;
+                if (!wait_or_abort(&sm.empty[s], (round & 1) ^ 1, sm.abort, wait_limit)) break;
                 tc::mbar_arrive_expect_tx(&sm.full[s], A_BYTES + C_BYTES);
                 tc::tma_load_2d(sm.a + s * A_BYTES, &tmap_a, &sm.full[s], kb * BK, m0);
                 tc::tma_load_2d(sm.c + s * C_BYTES, &tmap_c, &sm.full[s], kb * (BK / 16), n0);
@@ -166,18 +174,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // Drain: let every copy this thread started land before the CTA exits.
                 int zero = 0;
                 for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
-                    tc::mbar_wait_bounded(&sm.full[kb % STAGES], (kb / STAGES) & 1, &zero, kWaitCycles);
+                    tc::mbar_wait_bounded(&sm.full[kb % STAGES], (kb / STAGES) & 1, &zero, wait_limit);
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_i8(BM, BN);
-            for (int kb = 0; kb < num_kb; ++kb) {
+            if (stall) wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook: always times out
+            for (int kb = 0; kb < num_kb && !*reinterpret_cast<volatile int*>(sm.abort); ++kb) {
                 const int s = kb % STAGES;
                 const uint32_t parity = (kb / STAGES) & 1;
-                if (!wait_or_abort(&sm.full[s], parity, sm.abort)) break;
-                if (!wait_or_abort(&sm.decoded[s], parity, sm.abort)) break;
+                if (!wait_or_abort(&sm.full[s], parity, sm.abort, wait_limit)) break;
+                if (!wait_or_abort(&sm.decoded[s], parity, sm.abort, wait_limit)) break;
                 tc::tc_fence_after();
                 const uint32_t a_addr = tc::smem_u32(sm.a + s * A_BYTES);
                 const uint32_t b_addr = tc::smem_u32(sm.b + s * B_BYTES);
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % STAGES;
             const uint32_t parity = (kb / STAGES) & 1;
-            if (!wait_or_abort(&sm.full[s], parity, sm.abort)) break;
+            if (!wait_or_abort(&sm.full[s], parity, sm.abort, wait_limit)) break;
             const uint8_t* ctile = sm.c + s * C_BYTES;
             uint8_t* btile = sm.b + s * B_BYTES;
 #pragma unroll
@@ -217,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_arrive(&sm.decoded[s]);
         }
         // ---------------------------------------------------------------- epilogue
-        bool ok = wait_or_abort(sm.accum, 0, sm.abort) && !*reinterpret_cast<volatile int*>(sm.abort);
+        bool ok = wait_or_abort(sm.accum, 0, sm.abort, wait_limit) && !*reinterpret_cast<volatile int*>(sm.abort);
         ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective: decide per warp
         if (ok) {
             tc::tc_fence_after();
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Every MMA this CTA issued has been committed to sm.accum; make sure they are done.
         __syncwarp();
         int zero = 0;
-        tc::mbar_wait_bounded(sm.accum, 0, &zero, kWaitCycles);
+        tc::mbar_wait_bounded(sm.accum, 0, &zero, wait_limit);
         __syncwarp();
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem_d, TMEM_COLS);
@@ -295,11 +304,13 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(w2a4_gemm_kernel<OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    const cudaError_t e = ensure_smem(w2a4_gemm_kernel<OutT>, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((T + BM - 1) / BM));
-    w2a4_gemm_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(ma, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y);
+    const int stall = g_stall_next ? 1 : 0;
+    g_stall_next = false;
+    w2a4_gemm_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(ma, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
+                                                              g_wait_limit, stall);
     return cudaGetLastError();
 }
 
@@ -317,6 +328,9 @@ cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t
     if (f16) return gemm::launch_t<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
     return gemm::launch_t<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
 }
+
+void debug_set_gemm_wait_limit(long long cycles) { gemm::g_wait_limit = cycles > 0 ? cycles : gemm::kWaitCycles; }
+void debug_stall_next_gemm() { gemm::g_stall_next = true; }
 
 cudaError_t read_and_clear_device_error(int* word) {
     int v = 0;

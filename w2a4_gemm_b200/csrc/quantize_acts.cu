@@ -139,9 +139,8 @@ static cudaError_t launch_qa(const __half* x, int64_t tokens, int64_t K, int8_t*
         using S = FwhtShape<LOGB>;
         if (S::W > 1) smem += (size_t)(kActThreads / S::TPS) * S::B * sizeof(float);
     }
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(quant_acts_kernel<LOGB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = ensure_smem(quant_acts_kernel<LOGB>, smem);
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};

@@ -157,9 +157,8 @@ template <int SET>
 static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
                              uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
     const size_t smem = (size_t)n_in * sizeof(float);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(quant_weights_kernel<SET>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = ensure_smem(quant_weights_kernel<SET>, smem);
         if (e != cudaSuccess) return e;
     }
     quant_weights_kernel<SET><<<(unsigned)n_out, kQwThreads, smem, s>>>(w, n_in, G, lo, hi, codes, scales, row_mse);

@@ -49,9 +49,8 @@ static cudaError_t launch_rotate_t(const T* x, T* y, int64_t n_segments, float c
     const int64_t blocks = (n_segments + SPC - 1) / SPC;
     if (blocks > 0x7fffffff) return cudaErrorInvalidValue;
     if (blocks == 0) return cudaSuccess;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(rotate_kernel<LOGB, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+    {
+        const cudaError_t e = ensure_smem(rotate_kernel<LOGB, T>, smem);
         if (e != cudaSuccess) return e;
     }
     rotate_kernel<LOGB, T><<<(unsigned)blocks, kRotThreads, smem, s>>>(x, y, n_segments, c);
