@@ -202,3 +202,31 @@ def test_linear_gemm_parity(name, T, N, K):
         assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
                               ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32))
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
+# ------------------------------------------------------- every kernel family, same inputs
+@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm"])
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("T,N,K", [(1, 300, 4096), (2, 129, 512), (7, 64, 1024), (9, 257, 14336), (16, 4096, 4096),
+                                    (16, 130, 64), (5, 1000, 11008)])
+def test_linear_each_kernel_family(path, name, T, N, K):
+    qg.qift_debug_set_linear_path(path)
+    try:
+        for out_dtype in (torch.float16, torch.float32):
+            got, ref = _linear_case(name, T, N, K, 31 * T + N + K, out_dtype)
+            assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
+                                  ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32)), (path, T, N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
+def test_pinned_family_rejects_unsupported_shape():
+    qg.qift_debug_set_linear_path("skinny")
+    try:
+        q = torch.zeros((17, 64), dtype=torch.int8, device="cuda")
+        with pytest.raises(qg.QiftError):
+            qg.qift_linear(q, torch.ones(17, device="cuda"), torch.zeros((8, 4), dtype=torch.int32, device="cuda"),
+                           torch.ones(8, device="cuda"), "qift")
+    finally:
+        qg.qift_debug_set_linear_path("auto")

@@ -49,10 +49,12 @@ def lib() -> C.CDLL:
         L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
         L.qift_debug_set_wait_limit.argtypes = [i64]
         L.qift_debug_stall_next_gemm.argtypes = []
+        L.qift_debug_set_linear_path.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear",
-                     "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm"):
+                     "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
+                     "qift_debug_set_linear_path"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -169,3 +171,12 @@ def qift_debug_set_wait_limit(cycles: int) -> None:
 def qift_debug_stall_next_gemm() -> None:
     """Test hook: the next tensor-core GEMM waits on a barrier nothing arrives on and times out."""
     _check(lib().qift_debug_stall_next_gemm(), "qift_debug_stall_next_gemm")
+
+
+LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3}
+
+
+def qift_debug_set_linear_path(path) -> None:
+    """Test hook: pin qift_linear's kernel family ("auto", "gemv", "skinny", "gemm")."""
+    p = LINEAR_PATHS[path] if isinstance(path, str) else int(path)
+    _check(lib().qift_debug_set_linear_path(p), "qift_debug_set_linear_path")

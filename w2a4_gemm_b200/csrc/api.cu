@@ -27,6 +27,10 @@ bool valid_block(int64_t b) { return is_pow2(b) && b >= 2 && b <= 4096; }
 
 namespace qift {
 
+static int g_linear_path = kPathAuto;
+void debug_set_linear_path(int path) { g_linear_path = path; }
+int debug_linear_path() { return g_linear_path; }
+
 cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes) {
     static std::mutex mu;
     static std::unordered_map<uint64_t, size_t> granted;  // (kernel, device) -> bytes allowed
@@ -103,9 +107,24 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
         return QIFT_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f16 = out_dt == QIFT_F16;
-    if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
+    int path = qift::debug_linear_path();
+    if (path == qift::kPathAuto) {
+        if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
+            path = qift::kPathGemm;
+        else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
+            path = qift::kPathSkinny;
+        else
+            path = qift::kPathGemv;
+    } else if ((path == qift::kPathGemm && !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
+               (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))) {
+        return QIFT_ERR_UNSUPPORTED;
+    }
+    if (path == qift::kPathGemm)
         return from_cuda(qift::launch_linear_gemm(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y,
                                                   f16, s));
+    if (path == qift::kPathSkinny)
+        return from_cuda(qift::launch_linear_skinny(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in,
+                                                    y, f16, s));
     return from_cuda(
         qift::launch_linear_gemv(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y, f16, s));
 }
@@ -121,6 +140,12 @@ qift_status qift_device_error(void* stream, int32_t* detail) {
 
 qift_status qift_debug_set_wait_limit(int64_t cycles) {
     qift::debug_set_gemm_wait_limit((long long)cycles);
+    return QIFT_OK;
+}
+
+qift_status qift_debug_set_linear_path(int32_t path) {
+    if (path < 0 || path > 3) return QIFT_ERR_INVALID_ARG;
+    qift::debug_set_linear_path(path);
     return QIFT_OK;
 }
 

@@ -33,6 +33,12 @@ cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t
                                int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                cudaStream_t s);
 
+// Small-batch linear (<= 16 tokens): mma.sync skinny GEMM, cluster split-K over DSMEM.
+bool linear_skinny_supported(int64_t tokens, int64_t n_out, int64_t n_in);
+cudaError_t launch_linear_skinny(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                 int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
+                                 cudaStream_t s);
+
 // Prefill-size linear: tcgen05 int8 tensor-core GEMM with in-register code decode.
 bool linear_gemm_supported(int64_t tokens, int64_t n_out, int64_t n_in);
 cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
@@ -40,6 +46,9 @@ cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t
                                cudaStream_t s);
 
 // Test hooks behind qift_debug.h.
+enum LinearPath { kPathAuto = 0, kPathGemv = 1, kPathSkinny = 2, kPathGemm = 3 };
+void debug_set_linear_path(int path);
+int debug_linear_path();
 void debug_set_gemm_wait_limit(long long cycles);
 void debug_stall_next_gemm();
 

@@ -7,8 +7,10 @@
 //
 //   y[t][n] = ((float)acc[t][n] * s_w[n]) * s_a[t],  acc = sum_k q[t][k] * L(code[n][k]).
 //
-// One CTA computes a 128-token x 256-output tile, walking K in 128-byte blocks through a
-// 3-stage shared-memory ring:
+// One CTA computes a 128-token x 256-output tile, walking K in 128-byte blocks.  Two rings of
+// shared memory: STAGES slots for what TMA brings (the int8 activation tile and the packed
+// code tile), deep enough to cover the L2/HBM round trip, and BSTAGES slots for the decoded
+// int8 weight tile, which only has to run ahead of the tensor core by one block:
 //   warp 0      TMA producer: the int8 activation tile (128 x 128 B, 128-byte swizzle) and the
 //               packed code tile (256 rows x 8 words) land on one mbarrier per stage;
 //   warps 2..5  decoders: expand 2-bit codes to int8 weights in registers (byte permutes
@@ -34,12 +36,13 @@ namespace gemm {
 constexpr int BM = 128;          // tokens per tile (MMA M, TMEM lanes)
 constexpr int BN = 256;          // output features per tile (MMA N, TMEM columns)
 constexpr int BK = 128;          // K bytes per stage (one 128-byte swizzle row)
-constexpr int STAGES = 3;
+constexpr int STAGES = 6;        // TMA ring (activations + codes)
+constexpr int BSTAGES = 2;       // decoded-weight ring
 constexpr int kThreads = 192;    // 6 warps
 constexpr int A_BYTES = BM * BK;             // 16 KB
 constexpr int B_BYTES = BN * BK;             // 32 KB
 constexpr int C_BYTES = BN * (BK / 16) * 4;  // 8 KB of packed codes
-constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + C_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + C_BYTES) + BSTAGES * B_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 256;
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz before a wait gives up
 
@@ -52,9 +55,10 @@ struct Smem {
     uint8_t* a;
     uint8_t* b;
     uint8_t* c;
-    uint64_t* full;
-    uint64_t* decoded;
-    uint64_t* empty;
+    uint64_t* full;     // [STAGES]  TMA landed
+    uint64_t* empty;    // [STAGES]  MMA done with the slot
+    uint64_t* decoded;  // [BSTAGES] decoded weights written
+    uint64_t* bempty;   // [BSTAGES] MMA done with the decoded weights
     uint64_t* accum;
     uint64_t* never;
     uint32_t* tmem_base;
@@ -66,14 +70,15 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     Smem s;
     s.a = base;
     s.b = s.a + STAGES * A_BYTES;
-    s.c = s.b + STAGES * B_BYTES;
+    s.c = s.b + BSTAGES * B_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(s.c + STAGES * C_BYTES);
     s.full = bars;
-    s.decoded = bars + STAGES;
-    s.empty = bars + 2 * STAGES;
-    s.accum = bars + 3 * STAGES;
-    s.never = bars + 3 * STAGES + 1;
-    s.tmem_base = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 2);
+    s.empty = bars + STAGES;
+    s.decoded = bars + 2 * STAGES;
+    s.bempty = bars + 2 * STAGES + BSTAGES;
+    s.accum = bars + 2 * STAGES + 2 * BSTAGES;
+    s.never = s.accum + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     return s;
 }
@@ -138,8 +143,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             tc::mbar_init(&sm.full[s], 1);
-            tc::mbar_init(&sm.decoded[s], 128);
             tc::mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < BSTAGES; ++s) {
+            tc::mbar_init(&sm.decoded[s], 4);  // one arrive per decoder warp
+            tc::mbar_init(&sm.bempty[s], 1);
         }
         tc::mbar_init(sm.accum, 1);
         tc::mbar_init(sm.never, 1);
@@ -183,36 +191,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = tc::idesc_i8(BM, BN);
             if (stall) wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook: always times out
             for (int kb = 0; kb < num_kb && !*reinterpret_cast<volatile int*>(sm.abort); ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t parity = (kb / STAGES) & 1;
-                if (!wait_or_abort(&sm.full[s], parity, sm.abort, wait_limit)) break;
-                if (!wait_or_abort(&sm.decoded[s], parity, sm.abort, wait_limit)) break;
+                const int s = kb % STAGES, sb = kb % BSTAGES;
+                if (!wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit)) break;
+                if (!wait_or_abort(&sm.decoded[sb], (kb / BSTAGES) & 1, sm.abort, wait_limit)) break;
                 tc::tc_fence_after();
                 const uint32_t a_addr = tc::smem_u32(sm.a + s * A_BYTES);
-                const uint32_t b_addr = tc::smem_u32(sm.b + s * B_BYTES);
+                const uint32_t b_addr = tc::smem_u32(sm.b + sb * B_BYTES);
 #pragma unroll
                 for (int k = 0; k < BK / 32; ++k) {
                     tc::mma_i8_ss(tmem_d, tc::smem_desc_sw128(a_addr + 32 * k), tc::smem_desc_sw128(b_addr + 32 * k),
                                   idesc, (kb > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(&sm.empty[s]);
+                tc::mma_commit(&sm.bempty[sb]);
             }
             tc::mma_commit(sm.accum);  // also issued after an abort, so TMEM is idle before it is freed
         }
     } else {
         // ---------------------------------------------------------------- decoders
         const int d = threadIdx.x - 64;  // 0..127: rows d and d + 128 of the weight tile
+        // Rows r and r+4 of a quarter-warp would hit the same banks reading 32-byte code rows;
+        // every other group of four rows reads its second 16 bytes first.
+        const int first = (d >> 2) & 1;
         for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t parity = (kb / STAGES) & 1;
-            if (!wait_or_abort(&sm.full[s], parity, sm.abort, wait_limit)) break;
+            const int s = kb % STAGES, sb = kb % BSTAGES;
+            bool ok = wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit) &&
+                      wait_or_abort(&sm.bempty[sb], ((kb / BSTAGES) & 1) ^ 1, sm.abort, wait_limit);
+            if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together (it syncs below)
             const uint8_t* ctile = sm.c + s * C_BYTES;
-            uint8_t* btile = sm.b + s * B_BYTES;
+            uint8_t* btile = sm.b + sb * B_BYTES;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int r = d + 128 * h;
-                const uint4 w0 = *reinterpret_cast<const uint4*>(ctile + r * 32);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16);
+                const uint4 wa = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16 * first);
+                const uint4 wb = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16 * (first ^ 1));
+                const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
                 const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
                 uint8_t* brow = btile + r * BK;
 #pragma unroll
@@ -222,8 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
                 }
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&sm.decoded[s]);
+            tc::fence_proxy_async_smem();  // this lane's generic writes -> async proxy
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.decoded[sb]);
         }
         // ---------------------------------------------------------------- epilogue
         bool ok = wait_or_abort(sm.accum, 0, sm.abort, wait_limit) && !*reinterpret_cast<volatile int*>(sm.abort);

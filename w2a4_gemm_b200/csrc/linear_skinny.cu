@@ -1,0 +1,217 @@
+// linear_skinny.cu -- qift_linear for small batches (2..16 tokens): a tensor-core skinny GEMM
+// that streams the packed codes from HBM straight into mma fragments.
+//
+// "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+// Inference", Abstract: fixed 2-bit levels (Qift {+-1,+-3}, power-of-two {+-1,+-4}) applied to
+// 4-bit activations.  acc[t][n] = sum_k q[t][k] L(code[n][k]) in int32, then the fp32 scales.
+//
+// Work split.  A thread-block cluster of C CTAs shares one block of 128 output rows; CTA r of
+// the cluster owns the K slice [r*KS, (r+1)*KS).  Each of its 8 warps owns 16 rows.  The CTA
+// stages its slice of every token's int8 activations once in shared memory, permuted per
+// 16-byte group to the decode order, so the weights never touch shared memory: a lane loads
+// 16 bytes (4 words = 64 codes) of each of its two rows, decodes a word into four int8x4
+// registers with two masks, two shifts and four byte permutes against the level table, and
+// those registers ARE the A fragments of mma.m16n8k32 (s8 x s8 -> s32).  Partial int32 sums
+// of the C CTAs are added through distributed shared memory (exact, order-free), and the
+// cluster's CTAs each finish 128/C rows with the fp32 epilogue.  No global scratch.
+//
+// Fragment bookkeeping (g = lane/4, q = lane%4).  For chunk c (16 words of a row) and sub-step
+// j = 0..3, thread q handles word w = 16c + 4q + j of rows g and g+8; decode_word gives
+// d[0] = codes {0,2,4,6}, d[1] = {8,..,14}, d[2] = {1,3,5,7}, d[3] = {9,..,15} of w.  The MMA's
+// k-slots 4q..4q+3 / 16+4q..16+4q+3 are (d[0], d[1]) in the first MMA and (d[2], d[3]) in the
+// second; the B fragment of token g comes from the same activation group w, permuted the same
+// way.  Every thread pairs A and B on identical k positions, so the dot products are exact.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace qift {
+namespace skinny {
+
+namespace cg = cooperative_groups;
+
+constexpr int WARPS = 8;
+constexpr int RB = WARPS * 16;  // output rows per cluster
+constexpr int CHUNK_WORDS = 16;  // 256 K values per chunk
+
+__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Shared-memory slot of activation group G (16 bytes) within a token row: the low two bits
+// of G are XOR-ed with bits 2..3 so the four lanes of a quad and the next token row land on
+// distinct 16-byte bank groups.
+__device__ __forceinline__ int act_slot(int G) { return G ^ ((G >> 2) & 3); }
+
+template <typename OutT>
+__device__ __forceinline__ void store_y(OutT* p, float v);
+template <>
+__device__ __forceinline__ void store_y<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void store_y<__half>(__half* p, float v) { *p = __float2half_rn(v); }
+
+// NT token tiles of 8 (T <= 8*NT).  KS: K slice per CTA in bytes (multiple of 256).
+template <int NT, typename OutT>
+__global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __restrict__ q,
+                                                            const float* __restrict__ s_a,
+                                                            const uint32_t* __restrict__ codes,
+                                                            const float* __restrict__ s_w, uint32_t lut, int T,
+                                                            int N, int K, int KS, OutT* __restrict__ y) {
+    constexpr int TP = NT * 8;  // padded tokens
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int S = KS + 64;                            // token row stride (== 64 mod 128)
+    uint8_t* acts = smem;                             // TP x S bytes
+    int* part = reinterpret_cast<int*>(smem + TP * S);  // RB x TP int32 partial sums
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, qd = lane & 3;
+    const int row_block = blockIdx.x / C;
+    const int KW = K / 16;
+    const int kw0 = rank * (KS / 16);                  // first word of this CTA's slice
+    const int nchunks = KS / 256;
+    const int64_t r_lo = (int64_t)row_block * RB + warp * 16 + g;
+    const int64_t r_hi = r_lo + 8;
+
+    auto load_chunk = [&](int c, uint4& lo, uint4& hi) {
+        const int wi = kw0 + c * CHUNK_WORDS + 4 * qd;
+        lo = make_uint4(0u, 0u, 0u, 0u);
+        hi = make_uint4(0u, 0u, 0u, 0u);
+        if (wi + 4 <= KW) {
+            if (r_lo < N) lo = __ldg(reinterpret_cast<const uint4*>(codes + r_lo * KW + wi));
+            if (r_hi < N) hi = __ldg(reinterpret_cast<const uint4*>(codes + r_hi * KW + wi));
+        }
+    };
+
+    // Weights do not depend on the previous kernel: start streaming them before waiting.
+    uint4 cur_lo, cur_hi;
+    load_chunk(0, cur_lo, cur_hi);
+    griddep_launch_dependents();
+    griddep_wait();
+
+    // Stage this CTA's K slice of every token, permuted to the decode order.
+    const int groups = KS / 16;
+    for (int i = threadIdx.x; i < TP * groups; i += WARPS * 32) {
+        const int t = i / groups, G = i - t * groups;
+        const int64_t k = (int64_t)kw0 * 16 + (int64_t)G * 16;
+        uint4 a = make_uint4(0u, 0u, 0u, 0u);
+        if (t < T && k + 16 <= K) a = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
+        uint32_t p[4];
+        permute_acts(a, p);
+        *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+    __syncthreads();
+
+    int acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
+
+    for (int c = 0; c < nchunks; ++c) {
+        uint4 nxt_lo = make_uint4(0u, 0u, 0u, 0u), nxt_hi = make_uint4(0u, 0u, 0u, 0u);
+        if (c + 1 < nchunks) load_chunk(c + 1, nxt_lo, nxt_hi);
+        const uint32_t wl[4] = {cur_lo.x, cur_lo.y, cur_lo.z, cur_lo.w};
+        const uint32_t wh[4] = {cur_hi.x, cur_hi.y, cur_hi.z, cur_hi.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t dl[4], dh[4];
+            decode_word(wl[j], lut, dl);
+            decode_word(wh[j], lut, dh);
+            const uint32_t a1[4] = {dl[0], dh[0], dl[1], dh[1]};
+            const uint32_t a2[4] = {dl[2], dh[2], dl[3], dh[3]};
+            const int slot = act_slot(c * CHUNK_WORDS + 4 * qd + j);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
+                mma_s8(acc[nt], a1, p.x, p.y);
+                mma_s8(acc[nt], a2, p.z, p.w);
+            }
+        }
+        cur_lo = nxt_lo;
+        cur_hi = nxt_hi;
+    }
+
+    // Partial sums of this CTA's K slice: part[row][token].
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int rl = warp * 16 + g, t0 = nt * 8 + 2 * qd;
+        part[rl * TP + t0] = acc[nt][0];
+        part[rl * TP + t0 + 1] = acc[nt][1];
+        part[(rl + 8) * TP + t0] = acc[nt][2];
+        part[(rl + 8) * TP + t0 + 1] = acc[nt][3];
+    }
+    cluster.sync();
+
+    // CTA `rank` finishes rows [rank*RB/C, (rank+1)*RB/C) of the block: add the C partials.
+    const int rows_per = RB / C;
+    for (int i = threadIdx.x; i < rows_per * TP; i += WARPS * 32) {
+        const int rl = rank * rows_per + i / TP, t = i % TP;
+        int sum = 0;
+        for (int p = 0; p < C; ++p) {
+            const int* rp = cluster.map_shared_rank(part, p);
+            sum += rp[rl * TP + t];
+        }
+        const int64_t n = (int64_t)row_block * RB + rl;
+        if (t < T && n < N) {
+            const float v = __fmul_rn(__fmul_rn((float)sum, s_w[n]), s_a[t]);
+            store_y<OutT>(y + (int64_t)t * N + n, v);
+        }
+    }
+    cluster.sync();  // keep this CTA's partials alive until every peer has read them
+}
+
+template <int NT, typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    // Cluster size: enough K splits to spread small-N problems over the SMs, each slice at
+    // least two chunks.  C divides RB (so every CTA finishes a whole number of rows).
+    int C = 1;
+    while (C < 8 && K / (C * 2) >= 512) C *= 2;
+    const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
+    const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)RB * NT * 8 * sizeof(int);
+    cudaError_t e = ensure_smem(skinny_kernel<NT, OutT>, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t blocks = (N + RB - 1) / RB;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(blocks * C));
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N, (int)K, KS, y);
+}
+
+}  // namespace skinny
+
+bool linear_skinny_supported(int64_t T, int64_t N, int64_t K) {
+    return T >= 1 && T <= 16 && K % 64 == 0 && K <= 32768 && N <= (int64_t)0x7fffffff / 8;
+}
+
+cudaError_t launch_linear_skinny(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                                 int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (T <= 8) {
+        if (f16) return skinny::launch_t<1, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+        return skinny::launch_t<1, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+    }
+    if (f16) return skinny::launch_t<2, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return skinny::launch_t<2, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
+
+}  // namespace qift
