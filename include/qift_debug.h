@@ -25,6 +25,10 @@ qift_status qift_debug_set_wait_limit(int64_t cycles);
  * left unspecified and qift_device_error() then reports QIFT_ERR_TIMEOUT.  One-shot. */
 qift_status qift_debug_stall_next_gemm(void);
 
+/* Turn programmatic dependent launch of the decode-size kernels on (default) or off, to
+ * measure what the overlap with the previous kernel is worth.  Process-wide. */
+qift_status qift_debug_set_pdl(int32_t enable);
+
 /* Pin the kernel family qift_linear uses: 0 = automatic (by batch size), 1 = CUDA-core GEMV,
  * 2 = tensor-core skinny GEMM (tokens <= 16, n_in % 64 == 0), 3 = tcgen05 GEMM
  * (n_in % 64 == 0).  A pinned family that cannot take a call makes it return

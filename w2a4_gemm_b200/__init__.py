@@ -50,11 +50,12 @@ def lib() -> C.CDLL:
         L.qift_debug_set_wait_limit.argtypes = [i64]
         L.qift_debug_stall_next_gemm.argtypes = []
         L.qift_debug_set_linear_path.argtypes = [i32]
+        L.qift_debug_set_pdl.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
-                     "qift_debug_set_linear_path"):
+                     "qift_debug_set_linear_path", "qift_debug_set_pdl"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -180,3 +181,8 @@ def qift_debug_set_linear_path(path) -> None:
     """Test hook: pin qift_linear's kernel family ("auto", "gemv", "skinny", "gemm")."""
     p = LINEAR_PATHS[path] if isinstance(path, str) else int(path)
     _check(lib().qift_debug_set_linear_path(p), "qift_debug_set_linear_path")
+
+
+def qift_debug_set_pdl(enable: bool) -> None:
+    """Test hook: programmatic dependent launch of the decode kernels on (default) or off."""
+    _check(lib().qift_debug_set_pdl(1 if enable else 0), "qift_debug_set_pdl")

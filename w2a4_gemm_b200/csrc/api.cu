@@ -28,6 +28,9 @@ bool valid_block(int64_t b) { return is_pow2(b) && b >= 2 && b <= 4096; }
 namespace qift {
 
 static int g_linear_path = kPathAuto;
+static bool g_pdl = true;
+void debug_set_pdl(bool on) { g_pdl = on; }
+bool pdl_enabled() { return g_pdl; }
 void debug_set_linear_path(int path) { g_linear_path = path; }
 int debug_linear_path() { return g_linear_path; }
 
@@ -146,6 +149,11 @@ qift_status qift_debug_set_wait_limit(int64_t cycles) {
 qift_status qift_debug_set_linear_path(int32_t path) {
     if (path < 0 || path > 3) return QIFT_ERR_INVALID_ARG;
     qift::debug_set_linear_path(path);
+    return QIFT_OK;
+}
+
+qift_status qift_debug_set_pdl(int32_t enable) {
+    qift::debug_set_pdl(enable != 0);
     return QIFT_OK;
 }
 

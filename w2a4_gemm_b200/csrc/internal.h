@@ -49,6 +49,8 @@ cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t
 enum LinearPath { kPathAuto = 0, kPathGemv = 1, kPathSkinny = 2, kPathGemm = 3 };
 void debug_set_linear_path(int path);
 int debug_linear_path();
+void debug_set_pdl(bool on);
+bool pdl_enabled();  // programmatic dependent launch for the decode kernels (default on)
 void debug_set_gemm_wait_limit(long long cycles);
 void debug_stall_next_gemm();
 

@@ -13,10 +13,10 @@
 // int8 weight tile, which only has to run ahead of the tensor core by one block:
 //   warp 0      TMA producer: the int8 activation tile (128 x 128 B, 128-byte swizzle) and the
 //               packed code tile (256 rows x 8 words) land on one mbarrier per stage;
-//   warps 2..5  decoders: expand 2-bit codes to int8 weights in registers (byte permutes
-//               against the level table) and write them in the tensor core's 128-byte
-//               swizzled K-major layout; then, after the last block, the epilogue:
-//               tcgen05.ld of the int32 accumulators, the fp32 scale product, stores;
+//   warps 2..9  decoders (one weight row per thread): expand 2-bit codes to int8 weights in
+//               registers (byte permutes against the level table) and write them in the tensor
+//               core's 128-byte swizzled K-major layout; then, after the last block, the
+//               epilogue: tcgen05.ld of the int32 accumulators, the fp32 scale product, stores;
 //   warp 1      allocates 256 TMEM columns and one elected thread issues tcgen05.mma
 //               (kind::i8, M=128, N=256, K=32 per instruction, 4 per block), committing each
 //               stage back to the producer.
@@ -36,9 +36,10 @@ namespace gemm {
 constexpr int BM = 128;          // tokens per tile (MMA M, TMEM lanes)
 constexpr int BN = 256;          // output features per tile (MMA N, TMEM columns)
 constexpr int BK = 128;          // K bytes per stage (one 128-byte swizzle row)
-constexpr int STAGES = 6;        // TMA ring (activations + codes)
-constexpr int BSTAGES = 2;       // decoded-weight ring
-constexpr int kThreads = 192;    // 6 warps
+constexpr int STAGES = 5;        // TMA ring (activations + codes)
+constexpr int BSTAGES = 3;       // decoded-weight ring
+constexpr int kDecWarps = 8;     // one weight row of the tile per decoder thread
+constexpr int kThreads = 64 + 32 * kDecWarps;
 constexpr int A_BYTES = BM * BK;             // 16 KB
 constexpr int B_BYTES = BN * BK;             // 32 KB
 constexpr int C_BYTES = BN * (BK / 16) * 4;  // 8 KB of packed codes
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mbar_init(&sm.empty[s], 1);
         }
         for (int s = 0; s < BSTAGES; ++s) {
-            tc::mbar_init(&sm.decoded[s], 4);  // one arrive per decoder warp
+            tc::mbar_init(&sm.decoded[s], kDecWarps);  // one arrive per decoder warp
             tc::mbar_init(&sm.bempty[s], 1);
         }
         tc::mbar_init(sm.accum, 1);
@@ -209,31 +210,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- decoders
-        const int d = threadIdx.x - 64;  // 0..127: rows d and d + 128 of the weight tile
+        const int r = threadIdx.x - 64;  // 0..255: this thread's row of the weight tile
         // Rows r and r+4 of a quarter-warp would hit the same banks reading 32-byte code rows;
         // every other group of four rows reads its second 16 bytes first.
-        const int first = (d >> 2) & 1;
+        const int first = (r >> 2) & 1;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % STAGES, sb = kb % BSTAGES;
             bool ok = wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit) &&
                       wait_or_abort(&sm.bempty[sb], ((kb / BSTAGES) & 1) ^ 1, sm.abort, wait_limit);
             if (!__all_sync(0xffffffffu, ok)) break;  // the whole warp leaves together (it syncs below)
-            const uint8_t* ctile = sm.c + s * C_BYTES;
-            uint8_t* btile = sm.b + sb * B_BYTES;
+            const uint8_t* crow = sm.c + s * C_BYTES + r * 32;
+            const uint4 wa = *reinterpret_cast<const uint4*>(crow + 16 * first);
+            const uint4 wb = *reinterpret_cast<const uint4*>(crow + 16 * (first ^ 1));
+            const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint8_t* brow = sm.b + sb * B_BYTES + r * BK;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = d + 128 * h;
-                const uint4 wa = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16 * first);
-                const uint4 wb = *reinterpret_cast<const uint4*>(ctile + r * 32 + 16 * (first ^ 1));
-                const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
-                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                uint8_t* brow = btile + r * BK;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t v[4];
-                    decode_word_natural(words[c], lut, v);
-                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
-                }
+            for (int c = 0; c < 8; ++c) {
+                uint32_t v[4];
+                decode_word_natural(words[c], lut, v);
+                *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             tc::fence_proxy_async_smem();  // this lane's generic writes -> async proxy
             __syncwarp();
@@ -245,10 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             tc::tc_fence_after();
             const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
+            const int half = (warp - 2) >> 2;         // warps 2..5: columns 0..127, 6..9: 128..255
             const int row = m0 + quarter * 32 + lane;  // token
             const float sa = row < T ? s_a[row] : 0.0f;
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 16; ++cc) {
+            for (int cc = half * (BN / 32); cc < (half + 1) * (BN / 32); ++cc) {
                 uint32_t acc[16];
                 tc::tmem_ld_32x32b_x16(tmem_d + ((uint32_t)(quarter * 32) << 16) + cc * 16, acc);
                 tc::tmem_ld_wait();

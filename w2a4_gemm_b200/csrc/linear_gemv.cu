@@ -78,6 +78,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
     load_codes(0);
     griddep_launch_dependents();
     griddep_wait();
+    // Scales are requested now, so their latency hides under the code stream.
+    float sw[R], sa[TC];
+#pragma unroll
+    for (int r = 0; r < R; ++r) sw[r] = row0 + r < N ? __ldg(s_w + row0 + r) : 0.0f;
+#pragma unroll
+    for (int t = 0; t < TC; ++t) sa[t] = t0 + t < T ? __ldg(s_a + t0 + t) : 0.0f;
 
     for (int64_t base = 0; base < KW; base += 128 * J) {
         if (base > 0) load_codes(base);
@@ -127,7 +133,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
             const int sum = __reduce_add_sync(0xffffffffu, acc[r][t]);
             const int64_t n = row0 + r, tt = t0 + t;
             if (lane == ((r * TC + t) & 31) && n < N && tt < T) {
-                const float v = __fmul_rn(__fmul_rn((float)sum, s_w[n]), s_a[tt]);
+                const float v = __fmul_rn(__fmul_rn((float)sum, sw[r]), sa[t]);
                 store_out<OutT>(y + tt * N + n, v);
             }
         }
@@ -149,7 +155,7 @@ static cudaError_t launch_gemv_t(const int8_t* q, const float* s_a, const uint32
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     if ((K / 16) % 4 == 0)
         return cudaLaunchKernelEx(&cfg, gemv_kernel<TC, R, J, true, OutT>, q, s_a, codes, s_w, lut, T, N, K, y);
     return cudaLaunchKernelEx(&cfg, gemv_kernel<TC, R, J, false, OutT>, q, s_a, codes, s_w, lut, T, N, K, y);

@@ -34,6 +34,7 @@ namespace cg = cooperative_groups;
 constexpr int WARPS = 8;
 constexpr int RB = WARPS * 16;  // output rows per cluster
 constexpr int CHUNK_WORDS = 16;  // 256 K values per chunk
+constexpr int PF = 4;            // chunks of codes in flight per lane
 
 __device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -89,9 +90,11 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
         }
     };
 
-    // Weights do not depend on the previous kernel: start streaming them before waiting.
-    uint4 cur_lo, cur_hi;
-    load_chunk(0, cur_lo, cur_hi);
+    // Weights do not depend on the previous kernel: start streaming them before waiting.  A
+    // ring of PF chunks per lane keeps PF KB of codes per warp in flight.
+    uint4 buf[PF][2];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) load_chunk(u, buf[u][0], buf[u][1]);
     griddep_launch_dependents();
     griddep_wait();
 
@@ -114,28 +117,31 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
 
-    for (int c = 0; c < nchunks; ++c) {
-        uint4 nxt_lo = make_uint4(0u, 0u, 0u, 0u), nxt_hi = make_uint4(0u, 0u, 0u, 0u);
-        if (c + 1 < nchunks) load_chunk(c + 1, nxt_lo, nxt_hi);
-        const uint32_t wl[4] = {cur_lo.x, cur_lo.y, cur_lo.z, cur_lo.w};
-        const uint32_t wh[4] = {cur_hi.x, cur_hi.y, cur_hi.z, cur_hi.w};
+    for (int c0 = 0; c0 < nchunks; c0 += PF) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t dl[4], dh[4];
-            decode_word(wl[j], lut, dl);
-            decode_word(wh[j], lut, dh);
-            const uint32_t a1[4] = {dl[0], dh[0], dl[1], dh[1]};
-            const uint32_t a2[4] = {dl[2], dh[2], dl[3], dh[3]};
-            const int slot = act_slot(c * CHUNK_WORDS + 4 * qd + j);
+        for (int u = 0; u < PF; ++u) {
+            const int c = c0 + u;
+            if (c < nchunks) {
+                const uint32_t wl[4] = {buf[u][0].x, buf[u][0].y, buf[u][0].z, buf[u][0].w};
+                const uint32_t wh[4] = {buf[u][1].x, buf[u][1].y, buf[u][1].z, buf[u][1].w};
+                if (c + PF < nchunks) load_chunk(c + PF, buf[u][0], buf[u][1]);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
-                mma_s8(acc[nt], a1, p.x, p.y);
-                mma_s8(acc[nt], a2, p.z, p.w);
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t dl[4], dh[4];
+                    decode_word(wl[j], lut, dl);
+                    decode_word(wh[j], lut, dh);
+                    const uint32_t a1[4] = {dl[0], dh[0], dl[1], dh[1]};
+                    const uint32_t a2[4] = {dl[2], dh[2], dl[3], dh[3]};
+                    const int slot = act_slot(c * CHUNK_WORDS + 4 * qd + j);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
+                        mma_s8(acc[nt], a1, p.x, p.y);
+                        mma_s8(acc[nt], a2, p.z, p.w);
+                    }
+                }
             }
         }
-        cur_lo = nxt_lo;
-        cur_hi = nxt_hi;
     }
 
     // Partial sums of this CTA's K slice: part[row][token].
@@ -170,10 +176,11 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
 template <int NT, typename OutT>
 static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
                             int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
-    // Cluster size: enough K splits to spread small-N problems over the SMs, each slice at
-    // least two chunks.  C divides RB (so every CTA finishes a whole number of rows).
+    // Cluster size: split K so that each CTA streams a slice of at most 2048 inputs (64 KB of
+    // codes for its 128 rows) -- long-lived CTAs, yet enough of them when N is small.  C is a
+    // power of two <= 8, so it divides RB and every CTA finishes a whole number of rows.
     int C = 1;
-    while (C < 8 && K / (C * 2) >= 512) C *= 2;
+    while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
     const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
     const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)RB * NT * 8 * sizeof(int);
     cudaError_t e = ensure_smem(skinny_kernel<NT, OutT>, smem);
@@ -192,7 +199,7 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N, (int)K, KS, y);
 }
 

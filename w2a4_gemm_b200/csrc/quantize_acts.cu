@@ -152,7 +152,7 @@ static cudaError_t launch_qa(const __half* x, int64_t tokens, int64_t K, int8_t*
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, quant_acts_kernel<LOGB>, x, K, q, scales, c);
 }
 
