@@ -122,6 +122,24 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
                         const float* w_scale, qift_levelset set, int64_t tokens, int64_t n_out,
                         int64_t n_in, void* y, qift_dtype out_dt, void* stream);
 
+/*
+ * qift_decode_linear -- one decode step in a single launch: qift_quantize_acts followed by
+ * qift_linear, fused, for 1..4 tokens.  Same arithmetic and bit-identical results as the two
+ * calls; it exists because at decode batch sizes the separate activation kernel and the hand-off
+ * between the two launches cost more than the activation work itself.
+ *   x           : fp16 [tokens][n_in], 1 <= tokens <= 4; n_in % 64 == 0 and n_in <= 16384
+ *                 (other valid sizes return QIFT_ERR_UNSUPPORTED: use the two calls).
+ *   block       : Hadamard block as in qift_quantize_acts (0 = x already rotated).
+ *   codes, w_scale, set (QIFT or POT), n_out, y, out_dt: as in qift_linear.
+ *   q_out       : int8 [tokens][n_in] or NULL -- receives the INT4 activations.
+ *   act_scale_out: fp32 [tokens] or NULL -- receives s_a.
+ * Like the decode GEMV it may read `codes` before the kernel launched just before it on the
+ * same stream has finished, so that kernel must not write `codes`.
+ */
+qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int32_t block, const uint32_t* codes,
+                               const float* w_scale, qift_levelset set, int64_t n_out, void* y, qift_dtype out_dt,
+                               int8_t* q_out, float* act_scale_out, void* stream);
+
 /* qift_device_error -- synchronise `stream`, then read and clear the device error word.
  * Returns QIFT_OK, QIFT_ERR_TIMEOUT (a bounded on-chip wait gave up; that call's output is
  * invalid) or QIFT_ERR_CUDA.  *detail (may be NULL) receives the raw word. */

@@ -230,3 +230,40 @@ def test_pinned_family_rejects_unsupported_shape():
                            torch.ones(8, device="cuda"), "qift")
     finally:
         qg.qift_debug_set_linear_path("auto")
+
+
+# ---------------------------------------------------------- one-launch decode (fused a3-a5)
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("T,N,K,block", [(1, 4096, 4096, 4096), (1, 37, 64, 16), (2, 300, 512, 128), (3, 129, 11008, 128),
+                                          (4, 64, 14336, 128), (1, 1, 1024, 0), (4, 200, 2048, 2048), (1, 5000, 512, 512)])
+def test_decode_linear_matches_oracle(name, T, N, K, block):
+    rng = np.random.default_rng(T * 7 + N + K)
+    x = synth.activations(T, K, (T, N, K), n_outliers=synth.outlier_count(K))
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 16), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    q, s_a, _ = oracle.quantize_acts(x, block)
+    for out_dtype, npdt in ((torch.float16, np.float16), (torch.float32, np.float32)):
+        ref, _ = oracle.linear(q, s_a, codes, s_w, name, npdt)
+        gq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+        gsa = torch.empty(T, dtype=torch.float32, device="cuda")
+        gy = qg.qift_decode_linear(dev(x), block, dev(codes.view(np.int32)), dev(s_w), name, out_dtype,
+                                   q_out=gq, act_scale_out=gsa)
+        assert np.array_equal(host(gy).view(np.uint16 if npdt == np.float16 else np.uint32),
+                              ref.view(np.uint16 if npdt == np.float16 else np.uint32))
+        assert np.array_equal(host(gq), q)
+        assert np.array_equal(host(gsa).view(np.uint32), s_a.view(np.uint32))
+
+
+def test_decode_linear_zero_token_and_unsupported():
+    K, N = 256, 40
+    x = np.zeros((2, K), np.float16)
+    x[1] = synth.activations(1, K, (3,))[0]
+    rng = np.random.default_rng(0)
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 16), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    q, s_a, _ = oracle.quantize_acts(x, 64)
+    ref, _ = oracle.linear(q, s_a, codes, s_w, "qift", np.float32)
+    gy = qg.qift_decode_linear(dev(x), 64, dev(codes.view(np.int32)), dev(s_w), "qift", torch.float32)
+    assert np.array_equal(host(gy), ref)
+    with pytest.raises(qg.QiftError):
+        qg.qift_decode_linear(dev(np.zeros((5, K), np.float16)), 64, dev(codes.view(np.int32)), dev(s_w))

@@ -46,6 +46,7 @@ def lib() -> C.CDLL:
         L.qift_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
         L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
         L.qift_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, i32, vp]
+        L.qift_decode_linear.argtypes = [vp, i64, i64, i32, vp, vp, i32, i64, vp, i32, vp, vp, vp]
         L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
         L.qift_debug_set_wait_limit.argtypes = [i64]
         L.qift_debug_stall_next_gemm.argtypes = []
@@ -53,7 +54,7 @@ def lib() -> C.CDLL:
         L.qift_debug_set_pdl.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
-        for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear",
+        for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
                      "qift_debug_set_linear_path", "qift_debug_set_pdl"):
             getattr(L, name).restype = C.c_int
@@ -154,6 +155,28 @@ def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w
     dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
     _check(lib().qift_linear(_ptr(q), _ptr(act_scale), _ptr(codes), _ptr(w_scale), _set(levelset), T, N, K,
                              _ptr(y), dt, _stream(stream)), "qift_linear")
+    return y
+
+
+def qift_decode_linear(x: torch.Tensor, block: int, codes: torch.Tensor, w_scale: torch.Tensor, levelset="qift",
+                       out_dtype=torch.float16, out: torch.Tensor | None = None, q_out: torch.Tensor | None = None,
+                       act_scale_out: torch.Tensor | None = None, stream=None):
+    """One-launch decode step (1..4 tokens): rotation + INT4 + W2A4 linear.  Returns y."""
+    _cuda(x, "x", torch.float16)
+    _cuda(codes, "codes")
+    _cuda(w_scale, "w_scale", torch.float32)
+    T, K = x.shape
+    N = codes.shape[0]
+    if codes.shape[1] * 16 != K:
+        raise ValueError("codes must be [n_out, n_in/16]")
+    y = torch.empty((T, N), dtype=out_dtype, device=x.device) if out is None else _cuda(out, "out", out_dtype)
+    if q_out is not None:
+        _cuda(q_out, "q_out", torch.int8)
+    if act_scale_out is not None:
+        _cuda(act_scale_out, "act_scale_out", torch.float32)
+    dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
+    _check(lib().qift_decode_linear(_ptr(x), T, K, block, _ptr(codes), _ptr(w_scale), _set(levelset), N, _ptr(y), dt,
+                                    _ptr(q_out), _ptr(act_scale_out), _stream(stream)), "qift_decode_linear")
     return y
 
 

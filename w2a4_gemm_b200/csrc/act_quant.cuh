@@ -1,0 +1,125 @@
+// act_quant.cuh -- device pieces of the activation path shared by qift_quantize_acts and the
+// fused decode kernel: block Walsh-Hadamard rotation of one token into shared memory (fp32
+// stages, one rounding to fp16) with its max |x'|, and symmetric INT4 quantization.
+//
+// "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
+// Inference", Abstract: rotated W2A4 inference (4-bit activations).
+#pragma once
+
+#include "fwht.cuh"
+
+namespace qift {
+
+constexpr int kActThreads = 256;  // every function below needs all 256 threads of the CTA
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = lane < (kActThreads / 32) ? red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float m = red[0];
+    __syncthreads();  // red may be reused right after
+    return m;
+}
+
+// Shared memory the rotation needs besides the token itself (transpose buffer).
+template <int LOGB>
+__host__ __device__ constexpr size_t act_tbuf_bytes() {
+    if constexpr (LOGB == 0) {
+        return 0;
+    } else {
+        using S = FwhtShape<LOGB>;
+        return S::W > 1 ? (size_t)(kActThreads / S::TPS) * S::B * sizeof(float) : 0;
+    }
+}
+
+// Rotate one token (K fp16 values at xt, K % 16 == 0) into xs as fp16 and return max |x'|.
+// LOGB == 0: the token is already rotated (copied as is).  `red` holds kActThreads/32 floats.
+template <int LOGB>
+__device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt, int64_t K, float c, __half* xs,
+                                                  float* tbuf, float* red) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    float amax = 0.0f;
+    if constexpr (LOGB == 0) {
+        for (int64_t i = (int64_t)tid * 8; i < K; i += kActThreads * 8) {
+            const uint4 t = *reinterpret_cast<const uint4*>(xt + i);
+            *reinterpret_cast<uint4*>(xs + i) = t;
+            const __half2* h = reinterpret_cast<const __half2*>(&t);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(h[j]);
+                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    } else {
+        using S = FwhtShape<LOGB>;
+        constexpr int SPC = kActThreads / S::TPS;
+        const int seg_local = tid >> S::LOGT;
+        const int ts = tid & (S::TPS - 1);
+        const int64_t nseg = K / S::B;
+        for (int64_t p = 0; p < nseg; p += SPC) {
+            const int64_t seg = p + seg_local;
+            const bool active = seg < nseg;
+            float v[S::E];
+            if (active) {
+                load_contig<S::E>(xt + seg * S::B + ts * S::E, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < S::E; ++i) v[i] = 0.0f;
+            }
+            float out[S::W][S::R];
+            fwht_segment<LOGB>(v, ts, lane, c, tbuf + (S::W > 1 ? seg_local * S::B : 0), out);
+            if (active) {
+#pragma unroll
+                for (int j = 0; j < S::W; ++j) {
+                    float hv[S::R];
+#pragma unroll
+                    for (int r = 0; r < S::R; ++r) {
+                        hv[r] = __half2float(__float2half_rn(out[j][r]));
+                        amax = fmaxf(amax, fabsf(hv[r]));
+                    }
+                    store_contig<S::R>(xs + seg * S::B + ts * S::R + j * S::COL, hv);
+                }
+            }
+            if constexpr (S::W > 1) __syncthreads();  // tbuf is reused by the next pass
+        }
+    }
+    __syncthreads();
+    return block_max(amax, red);
+}
+
+// Sixteen fp16 values -> sixteen INT4 codes in int8 bytes, natural order:
+// clamp(rint_even(x * inv), -7, 7), one fp32 multiply per value.  inv = 7/m (IEEE division).
+__device__ __forceinline__ uint4 quant16(const __half* xs16, float inv) {
+    const uint4 a = *reinterpret_cast<const uint4*>(xs16);
+    const uint4 b = *reinterpret_cast<const uint4*>(xs16 + 8);
+    const __half2* ha = reinterpret_cast<const __half2*>(&a);
+    const __half2* hb = reinterpret_cast<const __half2*>(&b);
+    uint32_t packed[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const __half2* h = w < 2 ? ha + 2 * w : hb + 2 * (w - 2);
+        const float2 f0 = __half22float2(h[0]);
+        const float2 f1 = __half22float2(h[1]);
+        const float f[4] = {f0.x, f0.y, f1.x, f1.y};
+        uint32_t word = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int v = __float2int_rn(__fmul_rn(f[e], inv));
+            v = v > 7 ? 7 : (v < -7 ? -7 : v);
+            word |= (uint32_t)(v & 0xff) << (8 * e);
+        }
+        packed[w] = word;
+    }
+    return make_uint4(packed[0], packed[1], packed[2], packed[3]);
+}
+
+}  // namespace qift

@@ -132,6 +132,24 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
         qift::launch_linear_gemv(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y, f16, s));
 }
 
+qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int32_t block, const uint32_t* codes,
+                               const float* w_scale, qift_levelset set, int64_t n_out, void* y, qift_dtype out_dt,
+                               int8_t* q_out, float* act_scale_out, void* stream) {
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (out_dt != QIFT_F32 && out_dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
+    if (tokens < 0 || n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (block != 0 && (!valid_block(block) || n_in % block != 0)) return QIFT_ERR_INVALID_ARG;
+    if (set == QIFT_SET_STD || tokens > 4 || n_in > 16384 || n_in % 64 != 0) return QIFT_ERR_UNSUPPORTED;
+    if (tokens == 0 || n_out == 0) return QIFT_OK;
+    if (!x || !codes || !w_scale || !y) return QIFT_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(y) || !aligned4(w_scale)) return QIFT_ERR_INVALID_ARG;
+    if ((q_out && !aligned16(q_out)) || (act_scale_out && !aligned4(act_scale_out))) return QIFT_ERR_INVALID_ARG;
+    if (n_out > 0x7fffffff / 2) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(qift::launch_decode_linear(x, tokens, n_in, block, codes, w_scale, (int)set, n_out, y,
+                                                out_dt == QIFT_F16, q_out, act_scale_out,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 qift_status qift_device_error(void* stream, int32_t* detail) {
     if (detail) *detail = 0;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QIFT_ERR_CUDA;

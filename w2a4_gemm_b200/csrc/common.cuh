@@ -75,6 +75,17 @@ __device__ __forceinline__ void decode_word_natural(uint32_t w, uint32_t lut, ui
     d[3] = prmt(lut, 0u, hi >> 16);
 }
 
+// 16-byte read-only global load that the compiler keeps in program order relative to other
+// volatile asm (notably griddepcontrol.wait): used to put weight loads in flight before a
+// kernel waits for its predecessor.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // Programmatic dependent launch.  wait: block until the kernels this launch depends on have
 // completed and their writes are visible (a no-op without a programmatic dependency).
 // launch_dependents: allow the next kernel on the stream to start launching.

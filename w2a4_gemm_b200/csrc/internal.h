@@ -39,6 +39,11 @@ cudaError_t launch_linear_skinny(const int8_t* q, const float* s_a, const uint32
                                  int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                  cudaStream_t s);
 
+// One-launch decode step (1..4 tokens): rotation + INT4 + W2A4 GEMV, fused.
+cudaError_t launch_decode_linear(const void* x, int64_t tokens, int64_t n_in, int block, const uint32_t* codes,
+                                 const float* s_w, int set, int64_t n_out, void* y, bool f16, int8_t* q_out,
+                                 float* sa_out, cudaStream_t s);
+
 // Prefill-size linear: tcgen05 int8 tensor-core GEMM with in-register code decode.
 bool linear_gemm_supported(int64_t tokens, int64_t n_out, int64_t n_in);
 cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
                 if (n < N) {
                     const uint32_t* p = codes + n * KW + wi;
                     if (VEC && wi + 4 <= KW) {
-                        c = __ldg(reinterpret_cast<const uint4*>(p));
+                        c = ldg_stream_v4(p);
                     } else {
                         if (wi + 0 < KW) c.x = __ldg(p + 0);
                         if (wi + 1 < KW) c.y = __ldg(p + 1);

@@ -85,8 +85,8 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
         lo = make_uint4(0u, 0u, 0u, 0u);
         hi = make_uint4(0u, 0u, 0u, 0u);
         if (wi + 4 <= KW) {
-            if (r_lo < N) lo = __ldg(reinterpret_cast<const uint4*>(codes + r_lo * KW + wi));
-            if (r_hi < N) hi = __ldg(reinterpret_cast<const uint4*>(codes + r_hi * KW + wi));
+            if (r_lo < N) lo = ldg_stream_v4(codes + r_lo * KW + wi);
+            if (r_hi < N) hi = ldg_stream_v4(codes + r_hi * KW + wi);
         }
     };
 
