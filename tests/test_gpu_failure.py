@@ -34,8 +34,10 @@ def _case(T=128, N=256, K=512, seed=5):
     return args, ref
 
 
-def test_gemm_wait_timeout_is_reported_and_context_survives():
+@pytest.mark.parametrize("path", ["gemm", "gemm_ts"])
+def test_gemm_wait_timeout_is_reported_and_context_survives(path):
     args, ref = _case()
+    qg.qift_debug_set_linear_path(path)
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
     qg.qift_debug_set_wait_limit(20_000_000)          # ~10 ms per wait
     qg.qift_debug_stall_next_gemm()
@@ -48,3 +50,4 @@ def test_gemm_wait_timeout_is_reported_and_context_survives():
     torch.cuda.synchronize()
     assert np.array_equal(y.cpu().numpy(), ref)
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+    qg.qift_debug_set_linear_path("auto")

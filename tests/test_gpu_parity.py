@@ -192,20 +192,25 @@ def test_single_linear_256x512_end_to_end():
 
 
 # ------------------------------------------------------------- tensor-core GEMM (prefill)
+@pytest.mark.parametrize("path", ["gemm", "gemm_ts"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(17, 256, 64), (128, 256, 128), (129, 257, 192), (300, 600, 4096),
-                                    (256, 40, 640), (2048, 512, 11008), (64, 1000, 4160)])
-def test_linear_gemm_parity(name, T, N, K):
-    for out_dtype in (torch.float16, torch.float32):
-        got, ref = _linear_case(name, T, N, K, T + 7 * N + K, out_dtype)
-        tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
-        assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
-                              ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32))
+                                    (256, 40, 640), (2048, 512, 11008), (64, 1000, 4160), (513, 130, 1024)])
+def test_linear_gemm_parity(path, name, T, N, K):
+    qg.qift_debug_set_linear_path(path)
+    try:
+        for out_dtype in (torch.float16, torch.float32):
+            got, ref = _linear_case(name, T, N, K, T + 7 * N + K, out_dtype)
+            tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
+            assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
+                                  ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32))
+    finally:
+        qg.qift_debug_set_linear_path("auto")
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
 
 
 # ------------------------------------------------------- every kernel family, same inputs
-@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm", "gemm_ts"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(1, 300, 4096), (2, 129, 512), (7, 64, 1024), (9, 257, 14336), (16, 4096, 4096),
                                     (16, 130, 64), (5, 1000, 11008)])

@@ -327,6 +327,266 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 
 }  // namespace gemm
 
+// =====================================================================================
+// Variant with the decoded weights as the tensor core's A operand in TENSOR MEMORY.
+//
+// D[w][t] = sum_k W[w][k] * X[t][k]: the MMA's M = 128 weight rows (TMEM lanes), N = 256
+// tokens (TMEM columns).  Decoder threads own one weight row each; they expand its 128 codes of
+// a K block to int8 in 32 registers and write them with one tcgen05.st into that row's TMEM
+// lane -- the weights never touch shared memory, and per multiply-accumulate the decode work is
+// half that of the shared-memory variant (128 weight rows feed 256 tokens).  Shared memory only
+// carries what TMA brings: the activation tile (256 tokens x 128 B, 128-byte swizzle, the MMA's
+// B operand) and the packed codes (128 rows x 32 B).
+//   warp 0      TMA producer over a 6-stage ring
+//   warp 1      TMEM allocation (512 columns: accumulator 0..255, three A stages of 32 from
+//               256) and the single MMA-issuing thread (4 x K=32 per block)
+//   warps 2..9  two decoder groups of four warps (even / odd K blocks); afterwards, the epilogue
+//               (tcgen05.ld of D, scales, y[t][w] stores coalesced along w).
+// =====================================================================================
+namespace gemm_ts {
+
+constexpr int BMW = 128;                          // weight rows per tile (MMA M)
+constexpr int BNT = 256;                          // tokens per tile (MMA N)
+constexpr int BK = 128;                           // K bytes per block
+constexpr int STAGES = 6;                         // TMA ring
+constexpr int ASTAGES = 3;                        // decoded-weight stages in TMEM
+constexpr int kDecWarps = 8;
+constexpr int kThreads = 64 + 32 * kDecWarps;
+constexpr int ACT_BYTES = BNT * BK;               // 32 KB
+constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 4 KB
+constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t A_COL = 256;                   // A stage sa at A_COL + 32 * sa
+
+struct Smem {
+    uint8_t* act;
+    uint8_t* cod;
+    uint64_t* full;    // [STAGES]  TMA landed
+    uint64_t* empty;   // [STAGES]  MMA done with the slot
+    uint64_t* afull;   // [ASTAGES] decoded weights stored in TMEM
+    uint64_t* aempty;  // [ASTAGES] MMA done with the TMEM stage
+    uint64_t* accum;
+    uint64_t* never;
+    uint32_t* tmem_base;
+    int* abort;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    Smem s;
+    s.act = base;
+    s.cod = s.act + STAGES * ACT_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.cod + STAGES * COD_BYTES);
+    s.full = bars;
+    s.empty = bars + STAGES;
+    s.afull = bars + 2 * STAGES;
+    s.aempty = bars + 2 * STAGES + ASTAGES;
+    s.accum = bars + 2 * STAGES + 2 * ASTAGES;
+    s.never = s.accum + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
+    s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
+    return s;
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_one(OutT* p, float v);
+template <>
+__device__ __forceinline__ void store_one<float>(float* p, float v) { *p = v; }
+template <>
+__device__ __forceinline__ void store_one<__half>(__half* p, float v) { *p = __float2half_rn(v); }
+
+template <typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    w2a4_gemm_ts_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+                        const float* __restrict__ s_a, const float* __restrict__ s_w, uint32_t lut, int T, int N,
+                        int K, OutT* __restrict__ y, long long wait_limit, int stall) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BMW;   // first weight row
+    const int t0 = blockIdx.y * BNT;   // first token
+    const int num_kb = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < ASTAGES; ++s) {
+            tc::mbar_init(&sm.afull[s], 4);  // the four warps of one decoder group
+            tc::mbar_init(&sm.aempty[s], 1);
+        }
+        tc::mbar_init(sm.accum, 1);
+        tc::mbar_init(sm.never, 1);
+        *sm.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&tmap_x);
+        tc::prefetch_tensormap(&tmap_c);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *sm.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {  // ------------------------------------------------ TMA producer
+            int issued = 0;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const int s = kb % STAGES;
+                if (!gemm::wait_or_abort(&sm.empty[s], ((kb / STAGES) & 1) ^ 1, sm.abort, wait_limit)) break;
+                tc::mbar_arrive_expect_tx(&sm.full[s], ACT_BYTES + COD_BYTES);
+                tc::tma_load_2d(sm.act + s * ACT_BYTES, &tmap_x, &sm.full[s], kb * BK, t0);
+                tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.full[s], kb * (BK / 16), n0);
+                ++issued;
+            }
+            if (*reinterpret_cast<volatile int*>(sm.abort)) {
+                int zero = 0;  // drain: every copy this thread started lands before the CTA exits
+                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
+                    tc::mbar_wait_bounded(&sm.full[kb % STAGES], (kb / STAGES) & 1, &zero, wait_limit);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = tc::idesc_i8(BMW, BNT);
+            if (stall) gemm::wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook
+            for (int kb = 0; kb < num_kb && !*reinterpret_cast<volatile int*>(sm.abort); ++kb) {
+                const int s = kb % STAGES, sa = kb % ASTAGES;
+                if (!gemm::wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit)) break;
+                if (!gemm::wait_or_abort(&sm.afull[sa], (kb / ASTAGES) & 1, sm.abort, wait_limit)) break;
+                tc::tc_fence_after();
+                const uint32_t x_addr = tc::smem_u32(sm.act + s * ACT_BYTES);
+#pragma unroll
+                for (int k = 0; k < BK / 32; ++k)
+                    tc::mma_i8_ts(tmem + ACC_COL, tmem + A_COL + 32 * sa + 8 * k, tc::smem_desc_sw128(x_addr + 32 * k),
+                                  idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                tc::mma_commit(&sm.empty[s]);
+                tc::mma_commit(&sm.aempty[sa]);
+            }
+            tc::mma_commit(sm.accum);  // also after an abort, so TMEM is idle before it is freed
+        }
+    } else {
+        const int grp = (warp - 2) >> 2;      // decoder group: K blocks grp, grp + 2, ...
+        const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
+        const int r = quarter * 32 + lane;    // weight row of the tile
+        const int first = (r >> 2) & 1;       // staggered 16-byte halves: no bank conflicts
+        for (int kb = grp; kb < num_kb; kb += 2) {  // ---------------------- decoders
+            const int s = kb % STAGES, sa = kb % ASTAGES;
+            bool ok = gemm::wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit) &&
+                      gemm::wait_or_abort(&sm.aempty[sa], ((kb / ASTAGES) & 1) ^ 1, sm.abort, wait_limit);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc::tc_fence_after();
+            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 32;
+            const uint4 wa = *reinterpret_cast<const uint4*>(crow + 16 * first);
+            const uint4 wb = *reinterpret_cast<const uint4*>(crow + 16 * (first ^ 1));
+            const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t d[4];
+                decode_word_natural(words[c], lut, d);
+                v[4 * c] = d[0];
+                v[4 * c + 1] = d[1];
+                v[4 * c + 2] = d[2];
+                v[4 * c + 3] = d[3];
+            }
+            tc::tmem_st_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + 32 * sa, v);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.afull[sa]);
+        }
+        // ---------------------------------------------------------------- epilogue
+        bool ok = gemm::wait_or_abort(sm.accum, 0, sm.abort, wait_limit) &&
+                  !*reinterpret_cast<volatile int*>(sm.abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc::tc_fence_after();
+            const int n = n0 + r;
+            const float sw = n < N ? s_w[n] : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < BNT / 32; ++cc) {
+                const int c0 = grp * (BNT / 2) + cc * 16;  // token column within the tile
+                uint32_t acc[16];
+                tc::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
+                tc::tmem_ld_wait();
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = t0 + c0 + j;
+                        if (t < T) {
+                            const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), s_a[t]);
+                            store_one<OutT>(y + (int64_t)t * N + n, v);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        int zero = 0;
+        tc::mbar_wait_bounded(sm.accum, 0, &zero, wait_limit);
+        __syncwarp();
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    auto encode = gemm::get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap mx, mc;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {BK, BNT};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16) * 4};
+        const cuuint32_t box[2] = {BK / 16, BMW};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const cudaError_t e = ensure_smem(w2a4_gemm_ts_kernel<OutT>, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((N + BMW - 1) / BMW), (unsigned)((T + BNT - 1) / BNT));
+    const int stall = gemm::g_stall_next ? 1 : 0;
+    gemm::g_stall_next = false;
+    w2a4_gemm_ts_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
+                                                                 gemm::g_wait_limit, stall);
+    return cudaGetLastError();
+}
+
+}  // namespace gemm_ts
+
+cudaError_t launch_linear_gemm_ts(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                                  int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (f16) return gemm_ts::launch_t<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return gemm_ts::launch_t<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
+
 bool linear_gemm_supported(int64_t T, int64_t N, int64_t K) {
     // TMA needs 16-byte row strides for the code matrix (K % 64) and the grid fits.
     return K % 64 == 0 && T <= (int64_t)65535 * gemm::BM && N <= (int64_t)0x7fffffff;
