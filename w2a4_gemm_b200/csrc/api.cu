@@ -113,7 +113,7 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
     int path = qift::debug_linear_path();
     if (path == qift::kPathAuto) {
         if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
-            path = qift::kPathGemm;
+            path = qift::kPathGemmTs;
         else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
             path = qift::kPathSkinny;
         else
