@@ -8,6 +8,9 @@ Workloads (synthetic, seeded; shapes of LLaMA linear modules):
   decode16 LLaMA-3.1-8B MLP (gate/up 14336x4096, down 4096x14336), 16 tokens, 128-block, PoT
   prefill  LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008), 2048 tokens, 128-block, Qift
   single   one 256x512 linear, 8 tokens (parity case; timed for completeness)
+  offline  offline quantization of a full 8B-shaped model (224 modules, 6.98 G weights):
+           128-block rotation + per-row scale search + encode + pack for the Qift, PoT and
+           standard level sets; reports weights/s and the reconstruction MSE of each set
 
 A step is one online forward pass over one batch: qift_quantize_acts (rotation + INT4) and
 qift_linear for every linear of the workload.  The weights are quantized once, offline
@@ -399,13 +402,128 @@ def run_reference(args):
             "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ offline (8B-shaped model)
+ALU_EVAL_INSTR = 6  # compare, select, subtract, square, widen to fp64, fp64 add per candidate
+
+
+def alu_peak_evals(sm_mhz=1965.0, sms=148):
+    """Issue-bound peak of candidate evaluations per second: 4 schedulers x 32 lanes per SM."""
+    return sms * 4 * 32 * sm_mhz * 1e6 / ALU_EVAL_INSTR
+
+
+def run_offline(args, rank, world):
+    import torch
+    import w2a4_gemm_b200 as qg
+    from w2a4_gemm_b200 import build, synth
+    build.build()
+    qg.lib()
+    torch.cuda.set_device(rank % torch.cuda.device_count())
+    dev = torch.device("cuda")
+    mods = synth.model_8b_modules()
+    # Weights resident in HBM before timing (27.9 GB fp32), drawn on the device, seeded.
+    W = [synth.weights_t4_device(n_out, n_in, seed, dev) for (_, _, n_out, n_in, seed) in mods]
+    torch.cuda.synchronize()
+    biggest = max(w.numel() for w in W)
+    rot = torch.empty(biggest, dtype=torch.float32, device=dev)
+    codes = torch.empty(biggest // 16, dtype=torch.int32, device=dev)
+    scales = torch.empty(max(w.shape[0] for w in W), dtype=torch.float32, device=dev)
+    mse = {ls: [torch.empty(w.shape[0], dtype=torch.float64, device=dev) for w in W] for ls in ("qift", "pot", "std")}
+    L = qg.lib()
+    stream = qg._stream(None)
+
+    def step(_i):
+        for j, w in enumerate(W):
+            n_out, n_in = w.shape
+            r = rot[: w.numel()].view(n_out, n_in)
+            qg.qift_rotate(w, synth.MODEL_8B_BLOCK, out=r)
+            for ls in ("qift", "pot", "std"):
+                st = L.qift_quantize_weights(qg._ptr(r), n_out, n_in, qg.LEVELSETS[ls], 100, 0.2, 1.0,
+                                             qg._ptr(codes), qg._ptr(scales), qg._ptr(mse[ls][j]), stream)
+                qg._check(st, "qift_quantize_weights")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        s0.record()
+        for i in range(args.steps):
+            step(i)
+        e0.record()
+        torch.cuda.synchronize()
+        secs = max_over_ranks(s0.elapsed_time(e0) / 1e3, world)
+    clocks = clk.summary()
+    n_w = sum(w.numel() for w in W)
+    value = world * 3 * n_w * args.steps / secs
+    set_mse = {ls: float(sum((m * w.shape[1]).sum().item() for m, w in zip(mse[ls], W)) / n_w) for ls in mse}
+
+    # Live per-kernel timing of the two offline kernels on the largest module.
+    wbig = max(W, key=lambda w: w.numel())
+    n_out, n_in = wbig.shape
+    rb = rot[: wbig.numel()].view(n_out, n_in)
+    t_rot = time_region(torch, lambda i: qg.qift_rotate(wbig, synth.MODEL_8B_BLOCK, out=rb), 5) / 5
+    t_qw = time_region(torch, lambda i: L.qift_quantize_weights(qg._ptr(rb), n_out, n_in, 0, 100, 0.2, 1.0,
+                                                                qg._ptr(codes), qg._ptr(scales), None, stream), 3) / 3
+    evals = n_out * n_in * 100 / t_qw
+    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = alu_peak_evals(sm_mhz)
+    rot_b = 8 * wbig.numel()
+    return {
+        "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32+f64", "data": "synthetic",
+        "config": {"workload": "offline_8b_model_224_modules",
+                   "description": "rotate (128-block) + 100-point scale search + encode + pack of all 224 "
+                                  "linear modules of an 8B-shaped model, for each of the Qift, PoT and standard "
+                                  "level sets; Student-t(4)*0.02 weights drawn on the device",
+                   "weights": n_w, "level_sets": ["qift", "pot", "std"], "grid_points": 100,
+                   "l2": "inputs larger than L2 (27.9 GB of fp32 weights)",
+                   "reconstruction_mse": set_mse,
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": {"bound": "alu", "achieved": evals / 1e12, "peak": peak / 1e12, "unit": "T candidate-evals/s",
+                     "frac": evals / peak, "traffic": None, "kernel": "quant_weights_kernel (qift_quantize_weights)",
+                     "peak_source": f"issue-bound: 148 SMs x 128 lanes x {sm_mhz:.0f} MHz / {ALU_EVAL_INSTR} "
+                                    "instructions per candidate evaluation"},
+        "e2e": None, "gpu_launches": len(W) * 4 * args.steps, "clocks": clocks,
+        "stages": {"a1_rotate_weights": {"ms": t_rot * 1e3, "GB/s": rot_b / t_rot / 1e9,
+                                         "frac_hbm": rot_b / t_rot / 1e9 / peaks()["hbm_gbs"], "bound": "hbm"},
+                   "a2_quantize_weights": {"ms": t_qw * 1e3, "candidate_evals_per_s": evals, "bound": "alu",
+                                           "frac_alu": evals / peak}},
+    }
+
+
+def offline_cpu_baseline(budget_s=10.0):
+    """The oracle's rotate + quantize (three level sets) on a bounded sample of module rows."""
+    import oracle
+    from w2a4_gemm_b200 import synth
+    rows = 16
+    sample = [synth.weights(rows, n_in, (seed,)) for (_, _, _, n_in, seed) in synth.model_8b_modules()[:7]]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        for w in sample:
+            wr = oracle.rotate_f32(w, synth.MODEL_8B_BLOCK)
+            for ls in ("qift", "pot", "std"):
+                oracle.quantize_weights(wr, ls)
+            n += 3 * w.size
+        if time.perf_counter() - t0 > budget_s:
+            break
+    secs = time.perf_counter() - t0
+    return {"value": n / secs, "unit": "weights/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{rows} rows of each of the 7 projections of one layer, 3 level sets, repeated for "
+                      f"{secs:.1f} s"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single", "offline"], default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -423,9 +541,16 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", rank)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    line = run_ours(args, rank, world)
+    if args.workload == "offline":
+        line = run_offline(args, rank, world)
+    else:
+        line = run_ours(args, rank, world)
     if rank == 0:
-        line["cpu_baseline"] = cpu_baseline_obj(workload_def(args.workload), args.cpu_budget) if world == 1 else None
+        if world == 1:
+            line["cpu_baseline"] = (offline_cpu_baseline(args.cpu_budget) if args.workload == "offline"
+                                    else cpu_baseline_obj(workload_def(args.workload), args.cpu_budget))
+        else:
+            line["cpu_baseline"] = None
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

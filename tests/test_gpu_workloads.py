@@ -93,3 +93,20 @@ def test_offline_model_quantization_sampled(layer, proj):
         assert np.array_equal(host(gm)[rows].view(np.uint64), om.view(np.uint64))
         mse[ls] = host(gm).mean()
     assert mse["qift"] < mse["std"] and mse["pot"] < mse["std"]
+
+
+def test_offline_device_generated_module_parity():
+    # The offline benchmark draws the 8B-shaped model's weights on the device; the quantizer
+    # must match the oracle on those inputs too (sampled rows copied back to the host).
+    _, name, n_out, n_in, seed = synth.model_8b_modules()[7 * 5 + 6]   # layer 5 down_proj
+    W = synth.weights_t4_device(n_out, n_in, seed, "cuda")
+    w_rot = qg.qift_rotate(W, synth.MODEL_8B_BLOCK)
+    rows = np.sort(np.random.default_rng(seed).choice(n_out, size=24, replace=False))
+    Wh = host(W)[rows]
+    o_wrot = oracle.rotate_f32(Wh, synth.MODEL_8B_BLOCK)
+    assert np.array_equal(host(w_rot)[rows].view(np.uint32), o_wrot.view(np.uint32))
+    for ls in ("qift", "pot", "std"):
+        gc, gs, gm = qg.qift_quantize_weights(w_rot, ls)
+        oc, os_, om, _ = oracle.quantize_weights(o_wrot, ls)
+        assert np.array_equal(host(gc).view(np.uint32)[rows], oc)
+        assert np.array_equal(host(gm)[rows].view(np.uint64), om.view(np.uint64))

@@ -338,10 +338,11 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 // carries what TMA brings: the activation tile (256 tokens x 128 B, 128-byte swizzle, the MMA's
 // B operand) and the packed codes (128 rows x 32 B).
 //   warp 0      TMA producer over a 6-stage ring
-//   warp 1      TMEM allocation (512 columns: accumulator 0..255, three A stages of 32 from
+//   warp 1      TMEM allocation (512 columns: accumulator 0..255, five A stages of 32 from
 //               256) and the single MMA-issuing thread (4 x K=32 per block)
-//   warps 2..9  two decoder groups of four warps (even / odd K blocks); afterwards, the epilogue
-//               (tcgen05.ld of D, scales, y[t][w] stores coalesced along w).
+//   warps 2..17 four decoder groups of four warps (K blocks round-robin, so each group has four
+//               MMA periods for its decode); afterwards, the epilogue (tcgen05.ld of D, scales,
+//               y[t][w] stores coalesced along w).
 // =====================================================================================
 namespace gemm_ts {
 
@@ -349,12 +350,13 @@ constexpr int BMW = 128;                          // weight rows per tile (MMA M
 constexpr int BNT = 256;                          // tokens per tile (MMA N)
 constexpr int BK = 128;                           // K bytes per block
 constexpr int STAGES = 6;                         // TMA ring
-constexpr int ASTAGES = 3;                        // decoded-weight stages in TMEM
-constexpr int kDecWarps = 8;
+constexpr int ASTAGES = 5;                        // decoded-weight stages in TMEM
+constexpr int kGroups = 4;                        // decoder groups, K blocks round-robin
+constexpr int kDecWarps = 4 * kGroups;
 constexpr int kThreads = 64 + 32 * kDecWarps;
 constexpr int ACT_BYTES = BNT * BK;               // 32 KB
 constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 4 KB
-constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + 256;
+constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + 256 + BNT * 4 /*token scales*/;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t A_COL = 256;                   // A stage sa at A_COL + 32 * sa
@@ -370,6 +372,7 @@ struct Smem {
     uint64_t* never;
     uint32_t* tmem_base;
     int* abort;
+    float* sa;         // [BNT] activation scales of this tile's tokens
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
@@ -386,6 +389,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     s.never = s.accum + 1;
     s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
+    s.sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
     return s;
 }
 
@@ -427,6 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc::tmem_alloc(sm.tmem_base, TMEM_COLS);
         tc::tmem_relinquish();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + BNT) {
+        const int t = t0 + threadIdx.x - 64;
+        sm.sa[threadIdx.x - 64] = t < T ? s_a[t] : 0.0f;
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -470,11 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_commit(sm.accum);  // also after an abort, so TMEM is idle before it is freed
         }
     } else {
-        const int grp = (warp - 2) >> 2;      // decoder group: K blocks grp, grp + 2, ...
+        const int grp = (warp - 2) >> 2;      // decoder group: K blocks grp, grp + kGroups, ...
         const int quarter = warp & 3;         // TMEM lanes 32*quarter .. +31
         const int r = quarter * 32 + lane;    // weight row of the tile
         const int first = (r >> 2) & 1;       // staggered 16-byte halves: no bank conflicts
-        for (int kb = grp; kb < num_kb; kb += 2) {  // ---------------------- decoders
+        for (int kb = grp; kb < num_kb; kb += kGroups) {  // ---------------- decoders
             const int s = kb % STAGES, sa = kb % ASTAGES;
             bool ok = gemm::wait_or_abort(&sm.full[s], (kb / STAGES) & 1, sm.abort, wait_limit) &&
                       gemm::wait_or_abort(&sm.aempty[sa], ((kb / ASTAGES) & 1) ^ 1, sm.abort, wait_limit);
@@ -510,8 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = n0 + r;
             const float sw = n < N ? s_w[n] : 0.0f;
 #pragma unroll 1
-            for (int cc = 0; cc < BNT / 32; ++cc) {
-                const int c0 = grp * (BNT / 2) + cc * 16;  // token column within the tile
+            for (int cc = 0; cc < BNT / (16 * kGroups); ++cc) {
+                const int c0 = grp * (BNT / kGroups) + cc * 16;  // token column within the tile
                 uint32_t acc[16];
                 tc::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
                 tc::tmem_ld_wait();
@@ -520,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 16; ++j) {
                         const int t = t0 + c0 + j;
                         if (t < T) {
-                            const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), s_a[t]);
+                            const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[c0 + j]);
                             store_one<OutT>(y + (int64_t)t * N + n, v);
                         }
                     }

@@ -129,6 +129,20 @@ MODEL_8B_LAYERS = 32
 MODEL_8B_BLOCK = 128
 
 
+def weights_t4_device(n_out: int, n_in: int, seed: int, device, scale: float = 0.02):
+    """float32 [n_out, n_in] Student-t(4) * scale drawn ON the device (torch Philox generator):
+    t = z / sqrt(c / 4), z ~ N(0,1), c the sum of four squared N(0,1) draws.  Used where the
+    host generator would be too slow (the 6.98 G weights of the 8B-shaped model)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    z = torch.randn(n_out, n_in, generator=g, device=device)
+    c = torch.zeros(n_out, n_in, device=device)
+    for _ in range(4):
+        c.add_(torch.randn(n_out, n_in, generator=g, device=device).square_())
+    return z.mul_(torch.rsqrt(c.mul_(0.25))).mul_(scale)
+
+
 def model_8b_modules():
     """The 224 (layer, proj, n_out, n_in, seed) entries; seed = 1000 + 7*layer + proj index."""
     out = []
