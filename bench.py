@@ -429,7 +429,6 @@ def run_offline(args, rank, world):
     scales = torch.empty(max(w.shape[0] for w in W), dtype=torch.float32, device=dev)
     mse = {ls: [torch.empty(w.shape[0], dtype=torch.float64, device=dev) for w in W] for ls in ("qift", "pot", "std")}
     L = qg.lib()
-    stream = qg._stream(None)
 
     def step(_i):
         for j, w in enumerate(W):
@@ -438,7 +437,8 @@ def run_offline(args, rank, world):
             qg.qift_rotate(w, synth.MODEL_8B_BLOCK, out=r)
             for ls in ("qift", "pot", "std"):
                 st = L.qift_quantize_weights(qg._ptr(r), n_out, n_in, qg.LEVELSETS[ls], 100, 0.2, 1.0,
-                                             qg._ptr(codes), qg._ptr(scales), qg._ptr(mse[ls][j]), stream)
+                                             qg._ptr(codes), qg._ptr(scales), qg._ptr(mse[ls][j]),
+                                             qg._stream(None))
                 qg._check(st, "qift_quantize_weights")
 
     for i in range(args.warmup):
@@ -467,7 +467,8 @@ def run_offline(args, rank, world):
     rb = rot[: wbig.numel()].view(n_out, n_in)
     t_rot = time_region(torch, lambda i: qg.qift_rotate(wbig, synth.MODEL_8B_BLOCK, out=rb), 5) / 5
     t_qw = time_region(torch, lambda i: L.qift_quantize_weights(qg._ptr(rb), n_out, n_in, 0, 100, 0.2, 1.0,
-                                                                qg._ptr(codes), qg._ptr(scales), None, stream), 3) / 3
+                                                                qg._ptr(codes), qg._ptr(scales), None,
+                                                                qg._stream(None)), 3) / 3
     evals = n_out * n_in * 100 / t_qw
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
     peak = alu_peak_evals(sm_mhz)

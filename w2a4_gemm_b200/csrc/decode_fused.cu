@@ -6,8 +6,9 @@
 //
 // For 1..4 tokens the activation work is tiny next to streaming the packed weights, so every
 // CTA does it itself instead of waiting for a separate kernel:
-//   1. request this CTA's code rows (registers) -- before waiting for the previous kernel on
-//      the stream (programmatic dependent launch), so the weight stream overlaps its tail;
+//   1. load this CTA's code rows and decode them to int8 registers -- before waiting for the
+//      previous kernel on the stream (programmatic dependent launch), so the weight stream and
+//      the decode overlap its tail;
 //   2. rotate + quantize the tokens into shared memory (the same device code, and therefore
 //      the same bits, as qift_quantize_acts), stored permuted to the decode order;
 //   3. decode the codes to int8 (byte permutes against the level table) and dp4a them with the
@@ -25,7 +26,7 @@ namespace qift {
 namespace fused {
 
 constexpr int WARPS = kActThreads / 32;  // 8
-constexpr int RMAX = 4;                  // rows per warp
+constexpr int RMAX = 2;                  // rows per warp
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* p, float v);
@@ -57,21 +58,26 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
     const int64_t row0 = cta_r0 + (int64_t)warp * rpw;
     const int nr = (int)max((int64_t)0, min((int64_t)rpw, cta_r1 - row0));
 
-    uint4 cw[RMAX][J];
-    auto load_codes = [&](int64_t base) {
+    // Codes of the first K chunk are loaded and decoded to int8 registers before waiting for
+    // the previous kernel: only the activation work and the dp4a products remain after it.
+    uint32_t dec[RMAX][J][4][4];
+    auto load_decode = [&](int64_t base) {
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) {
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 const int64_t wi = base + 4 * lane + 128 * j;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (r < nr && wi + 4 <= KW) v = ldg_stream_v4(codes + (row0 + r) * KW + wi);
-                cw[r][j] = v;
+                const uint4 v = (r < nr && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
+                                                         : make_uint4(0u, 0u, 0u, 0u);
+                decode_word(v.x, lut, dec[r][j][0]);
+                decode_word(v.y, lut, dec[r][j][1]);
+                decode_word(v.z, lut, dec[r][j][2]);
+                decode_word(v.w, lut, dec[r][j][3]);
             }
         }
     };
     // 1. weights first, then wait for the producer of x.
-    load_codes(0);
+    load_decode(0);
     griddep_launch_dependents();
     griddep_wait();
     float sw[RMAX];
@@ -111,7 +117,7 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
 #pragma unroll
         for (int t = 0; t < TC; ++t) acc[r][t] = 0;
     for (int64_t base = 0; base < KW; base += 128 * J) {
-        if (base > 0) load_codes(base);
+        if (base > 0) load_decode(base);
         uint4 pa[TC][J][4];
 #pragma unroll
         for (int t = 0; t < TC; ++t)
@@ -128,18 +134,15 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
             if (r >= nr) break;
 #pragma unroll
             for (int j = 0; j < J; ++j) {
-                const uint32_t words[4] = {cw[r][j].x, cw[r][j].y, cw[r][j].z, cw[r][j].w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    uint32_t d[4];
-                    decode_word(words[u], lut, d);
 #pragma unroll
                     for (int t = 0; t < TC; ++t) {
                         int a = acc[r][t];
-                        a = dp4a(d[0], pa[t][j][u].x, a);
-                        a = dp4a(d[1], pa[t][j][u].y, a);
-                        a = dp4a(d[2], pa[t][j][u].z, a);
-                        a = dp4a(d[3], pa[t][j][u].w, a);
+                        a = dp4a(dec[r][j][u][0], pa[t][j][u].x, a);
+                        a = dp4a(dec[r][j][u][1], pa[t][j][u].y, a);
+                        a = dp4a(dec[r][j][u][2], pa[t][j][u].z, a);
+                        a = dp4a(dec[r][j][u][3], pa[t][j][u].w, a);
                         acc[r][t] = a;
                     }
                 }

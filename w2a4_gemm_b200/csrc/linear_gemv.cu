@@ -140,6 +140,105 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
     }
 }
 
+// One token, n_in % 64 == 0: the codes of the first K chunk are loaded AND decoded to int8
+// registers before the kernel waits for its predecessor, so after the wait only the
+// activation token (staged once per CTA in shared memory, permuted to the decode order), the
+// dp4a products, the warp reduction and the epilogue remain on the critical path.
+template <int R, int J, typename OutT>
+__global__ void __launch_bounds__(kGemvWarps * 32) gemv1_kernel(const int8_t* __restrict__ q,
+                                                                const float* __restrict__ s_a,
+                                                                const uint32_t* __restrict__ codes,
+                                                                const float* __restrict__ s_w, uint32_t lut,
+                                                                int64_t N, int64_t K, OutT* __restrict__ y) {
+    extern __shared__ __align__(16) uint4 acts_s[];  // K/16 permuted 16-byte groups
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (int64_t)blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
+    const int64_t row0 = warp * R;
+    const int64_t KW = K / 16;
+
+    uint32_t dec[R][J][4][4];
+    auto load_decode = [&](int64_t base) {
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int64_t wi = base + 4 * lane + 128 * j;
+                const uint4 c = (row0 + r < N && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
+                                                              : make_uint4(0u, 0u, 0u, 0u);
+                decode_word(c.x, lut, dec[r][j][0]);
+                decode_word(c.y, lut, dec[r][j][1]);
+                decode_word(c.z, lut, dec[r][j][2]);
+                decode_word(c.w, lut, dec[r][j][3]);
+            }
+        }
+    };
+    load_decode(0);
+    griddep_launch_dependents();
+    griddep_wait();
+
+    float sw[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) sw[r] = row0 + r < N ? __ldg(s_w + row0 + r) : 0.0f;
+    const float sa = __ldg(s_a);
+    for (int64_t i = threadIdx.x; i < KW; i += kGemvWarps * 32) {
+        uint32_t p[4];
+        permute_acts(__ldg(reinterpret_cast<const uint4*>(q) + i), p);
+        acts_s[i] = make_uint4(p[0], p[1], p[2], p[3]);
+    }
+    __syncthreads();
+
+    int acc[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = 0;
+    for (int64_t base = 0; base < KW; base += 128 * J) {
+        if (base > 0) load_decode(base);
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t wi = base + 4 * lane + 128 * j + u;
+                const uint4 a = wi < KW ? acts_s[wi] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    int v = acc[r];
+                    v = dp4a(dec[r][j][u][0], a.x, v);
+                    v = dp4a(dec[r][j][u][1], a.y, v);
+                    v = dp4a(dec[r][j][u][2], a.z, v);
+                    v = dp4a(dec[r][j][u][3], a.w, v);
+                    acc[r] = v;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int sum = __reduce_add_sync(0xffffffffu, acc[r]);
+        if (lane == r && row0 + r < N)
+            store_out<OutT>(y + row0 + r, __fmul_rn(__fmul_rn((float)sum, sw[r]), sa));
+    }
+}
+
+template <int R, int J, typename OutT>
+static cudaError_t launch_gemv1(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                uint32_t lut, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    const int64_t gx = ((N + R - 1) / R + kGemvWarps - 1) / kGemvWarps;
+    if (gx > 0x7fffffff) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)K;  // K/16 groups of 16 bytes
+    cudaError_t e = ensure_smem(gemv1_kernel<R, J, OutT>, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)gx);
+    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemv1_kernel<R, J, OutT>, q, s_a, codes, s_w, lut, N, K, y);
+}
+
 template <int TC, int R, int J, typename OutT>
 static cudaError_t launch_gemv_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                  uint32_t lut, int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
@@ -164,6 +263,7 @@ static cudaError_t launch_gemv_t(const int8_t* q, const float* s_a, const uint32
 template <typename OutT>
 static cudaError_t dispatch_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                  uint32_t lut, int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    if (T == 1 && K % 64 == 0) return launch_gemv1<2, 2, OutT>(q, s_a, codes, s_w, lut, N, K, y, s);
     if (T == 1) return launch_gemv_t<1, 4, 2, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
     if (T == 2) return launch_gemv_t<2, 4, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
     return launch_gemv_t<4, 2, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
