@@ -255,6 +255,12 @@ def run_ours(args, rank, world):
     t_lin = time_region(torch, lambda i: qg.qift_linear(L0["q"][i % copies], L0["sa"][i % copies],
                                                         L0["codes"][i % copies], L0["s_w"][i % copies], wl.levelset,
                                                         st.out_dt, out=L0["y"][i % copies]), reps) / reps
+    t_fused = None
+    if T <= 4 and lin0.n_in % 64 == 0 and lin0.n_in <= 16384 and wl.levelset != "std":
+        t_fused = time_region(torch, lambda i: qg.qift_decode_linear(L0["x"][i % copies], wl.a_block,
+                                                                     L0["codes"][i % copies], L0["s_w"][i % copies],
+                                                                     wl.levelset, st.out_dt, out=L0["y"][i % copies]),
+                              reps) / reps
     W, _ = st.offline[0]
     w_rot = torch.empty_like(W)
     t_rot = time_region(torch, lambda i: qg.qift_rotate(W, wl.w_block, out=w_rot), 5) / 5
@@ -276,6 +282,11 @@ def run_ours(args, rank, world):
                       "frac_hbm": lin_b / t_lin / 1e9 / pk["hbm_gbs"],
                       "frac_int8": 2 * T * N0 * K0 / t_lin / 1e12 / pk["int8_tops"]},
     }
+    if t_fused is not None:
+        fb = acts_bytes(T, K0) - T * K0 - 4 * T + lin_b - T * K0 - 4 * T  # x in, codes, scales, y out
+        stages["a3a4a5_fused_decode"] = {"ms": t_fused * 1e3, "bytes": fb, "GB/s": fb / t_fused / 1e9,
+                                         "frac_hbm": fb / t_fused / 1e9 / pk["hbm_gbs"], "bound": "hbm",
+                                         "entry": "qift_decode_linear (one launch)"}
 
     if decode:
         value = world * step_bytes * args.steps / secs / 1e9
