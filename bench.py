@@ -52,6 +52,38 @@ def peaks():
     return dict(hbm_gbs=hbm, int8_tops=2.0 * bf16, int8_tops_sustained=2.0 * bf16s, source=src)
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel,
+# from one ncu capture of the same workload (summaries in profiles/).  Each entry is keyed by a
+# hash of the kernel's sources; if they have changed since the capture the traffic is reported
+# as null.  `scale` converts the captured launch to the benchmarked one when the shapes differ
+# (traffic grows in proportion to the weights processed).
+PROFILED_TRAFFIC = {
+    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="ac7b33485df99f62", bytes=4231168 + 0,
+                   profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="8c6476ba935a999f",
+                    bytes=19738112 + 2433280, profile="profiles/w2a4_gemm_ts_kernel_mlp_prefill_T2048.md"),
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="cb37b8ef06a6c6db", bytes=14833152 + 0,
+                     profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
+    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="d77053b1a3d2c13a",
+                    bytes=67137024 + 690688, scale=14336 * 4096 / (4096 * 4096),
+                    profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
+}
+
+
+def profiled_traffic(workload):
+    import hashlib
+    e = PROFILED_TRAFFIC.get(workload)
+    if not e:
+        return None
+    h = hashlib.sha1()
+    for f in e["files"]:
+        with open(os.path.join(ROOT, "w2a4_gemm_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != e["sha"]:
+        return None
+    return e["bytes"] * e.get("scale", 1.0)
+
+
 # ----------------------------------------------------------------------------- workloads
 def workload_def(name):
     from w2a4_gemm_b200 import synth
@@ -292,14 +324,16 @@ def run_ours(args, rank, world):
         value = world * step_bytes * args.steps / secs / 1e9
         unit = "GB/s"
         roof = {"bound": "hbm", "achieved": lin_b / t_lin / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": lin_b / t_lin / 1e9 / pk["hbm_gbs"], "traffic": None, "kernel": "qift_linear (GEMV)",
+                "frac": lin_b / t_lin / 1e9 / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload),
+                "kernel": "qift_linear (GEMV)",
                 "peak_source": pk["source"] + " copy bandwidth, burst"}
     else:
         value = world * step_ops * args.steps / secs / 1e12
         unit = "TOPS"
         ach = 2 * T * N0 * K0 / t_lin / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": pk["int8_tops"], "unit": "TOPS",
-                "frac": ach / pk["int8_tops"], "traffic": None, "kernel": "qift_linear (GEMM)",
+                "frac": ach / pk["int8_tops"], "traffic": profiled_traffic(args.workload),
+                "kernel": "qift_linear (GEMM)",
                 "peak_source": pk["source"] + " bf16 burst x 2 (int8 nominal ratio)"}
 
     # End to end through the public API: pinned host x -> device, both calls, y -> pinned host.
@@ -497,7 +531,8 @@ def run_offline(args, rank, world):
                    "reconstruction_mse": set_mse,
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "roofline": {"bound": "alu", "achieved": evals / 1e12, "peak": peak / 1e12, "unit": "T candidate-evals/s",
-                     "frac": evals / peak, "traffic": None, "kernel": "quant_weights_kernel (qift_quantize_weights)",
+                     "frac": evals / peak, "traffic": profiled_traffic("offline"),
+                     "kernel": "quant_weights_kernel (qift_quantize_weights)",
                      "peak_source": f"issue-bound: 148 SMs x 128 lanes x {sm_mhz:.0f} MHz / {ALU_EVAL_INSTR} "
                                     "instructions per candidate evaluation"},
         "e2e": None, "gpu_launches": len(W) * 4 * args.steps, "clocks": clocks,
