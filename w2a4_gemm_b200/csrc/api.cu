@@ -118,11 +118,14 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
             path = qift::kPathSkinny;
         else
             path = qift::kPathGemv;
-    } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs) &&
+    } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs || path == qift::kPathGemmTsp) &&
                 !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
                (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))) {
         return QIFT_ERR_UNSUPPORTED;
     }
+    if (path == qift::kPathGemmTsp)
+        return from_cuda(qift::launch_linear_gemm_tsp(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
+                                                      n_in, y, f16, s));
     if (path == qift::kPathGemmTs)
         return from_cuda(qift::launch_linear_gemm_ts(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
                                                      n_in, y, f16, s));
@@ -169,7 +172,7 @@ qift_status qift_debug_set_wait_limit(int64_t cycles) {
 }
 
 qift_status qift_debug_set_linear_path(int32_t path) {
-    if (path < 0 || path > 4) return QIFT_ERR_INVALID_ARG;
+    if (path < 0 || path > 5) return QIFT_ERR_INVALID_ARG;
     qift::debug_set_linear_path(path);
     return QIFT_OK;
 }

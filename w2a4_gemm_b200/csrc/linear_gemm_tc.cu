@@ -24,6 +24,8 @@
 // the device error word, every role drains what it started, TMEM is freed and the CTA exits.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "tc.cuh"
 
@@ -586,6 +588,323 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 }
 
 }  // namespace gemm_ts
+
+// =====================================================================================
+// Persistent variant of the tensor-memory-A GEMM: one CTA per SM walks a list of
+// 128-weight-row x 128-token tiles.  Two accumulators in TMEM (columns 0..127 and 128..255)
+// let four dedicated epilogue warps drain tile i while the MMAs of tile i+1 run, and the TMA
+// ring and the decoders run straight on into the next tile, so no pipeline fill or epilogue
+// is exposed between tiles.
+//   warp 0        TMA producer (8-stage ring: 128 tokens x 128 B activations + 128 x 32 B codes)
+//   warp 1        TMEM owner and MMA issuer (M = 128 weight rows, N = 128 tokens)
+//   warps 2..17   decoders, four groups taking K blocks round-robin across tiles
+//   warps 18..21  epilogue: tcgen05.ld, scales, y stores; frees an accumulator per tile
+// =====================================================================================
+namespace gemm_tsp {
+
+constexpr int BMW = 128;
+constexpr int BNT = 128;
+constexpr int BK = 128;
+constexpr int STAGES = 8;
+constexpr int ASTAGES = 5;
+constexpr int kGroups = 4;
+constexpr int kDecWarps = 4 * kGroups;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + 32 * (kDecWarps + kEpiWarps);
+constexpr int ACT_BYTES = BNT * BK;               // 16 KB
+constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 4 KB
+constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + 512 + 2 * BNT * 4;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t A_COL = 2 * BNT;               // accumulators at 0 and BNT
+
+struct Smem {
+    uint8_t* act;
+    uint8_t* cod;
+    uint64_t* full;
+    uint64_t* empty;
+    uint64_t* afull;
+    uint64_t* aempty;
+    uint64_t* accfull;   // [2]
+    uint64_t* accempty;  // [2]
+    uint64_t* done;
+    uint64_t* never;
+    uint32_t* tmem_base;
+    int* abort;
+    float* sa;           // [2][BNT] token scales of the tile held in each accumulator
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    Smem s;
+    s.act = base;
+    s.cod = s.act + STAGES * ACT_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.cod + STAGES * COD_BYTES);
+    s.full = bars;
+    s.empty = s.full + STAGES;
+    s.afull = s.empty + STAGES;
+    s.aempty = s.afull + ASTAGES;
+    s.accfull = s.aempty + ASTAGES;
+    s.accempty = s.accfull + 2;
+    s.done = s.accempty + 2;
+    s.never = s.done + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
+    s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
+    s.sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
+    return s;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory"); }
+
+template <typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    w2a4_gemm_tsp_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+                         const float* __restrict__ s_a, const float* __restrict__ s_w, uint32_t lut, int T, int N,
+                         int K, OutT* __restrict__ y, long long wait_limit, int stall) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_kb = (K + BK - 1) / BK;
+    const int n_tiles_w = (N + BMW - 1) / BMW;
+    const int n_tiles = n_tiles_w * ((T + BNT - 1) / BNT);
+    const int my_tiles = blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < ASTAGES; ++s) {
+            tc::mbar_init(&sm.afull[s], 4);
+            tc::mbar_init(&sm.aempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&sm.accfull[b], 1);
+            tc::mbar_init(&sm.accempty[b], kEpiWarps);
+        }
+        tc::mbar_init(sm.done, 1);
+        tc::mbar_init(sm.never, 1);
+        *sm.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&tmap_x);
+        tc::prefetch_tensormap(&tmap_c);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *sm.tmem_base;
+    volatile int* abort_v = reinterpret_cast<volatile int*>(sm.abort);
+
+    if (warp == 0) {
+        if (lane == 0) {  // ------------------------------------------------ TMA producer
+            int g = 0, issued = 0;
+            for (int i = 0; i < my_tiles && !*abort_v; ++i) {
+                const int tile = blockIdx.x + i * gridDim.x;
+                const int n0 = (tile % n_tiles_w) * BMW, t0 = (tile / n_tiles_w) * BNT;
+                for (int kb = 0; kb < num_kb; ++kb, ++g) {
+                    const int s = g % STAGES;
+                    if (!gemm::wait_or_abort(&sm.empty[s], ((g / STAGES) & 1) ^ 1, sm.abort, wait_limit)) break;
+                    tc::mbar_arrive_expect_tx(&sm.full[s], ACT_BYTES + COD_BYTES);
+                    tc::tma_load_2d(sm.act + s * ACT_BYTES, &tmap_x, &sm.full[s], kb * BK, t0);
+                    tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.full[s], kb * (BK / 16), n0);
+                    ++issued;
+                }
+            }
+            if (*abort_v) {
+                int zero = 0;  // drain every copy this thread started
+                for (int q = issued > STAGES ? issued - STAGES : 0; q < issued; ++q)
+                    tc::mbar_wait_bounded(&sm.full[q % STAGES], (q / STAGES) & 1, &zero, wait_limit);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = tc::idesc_i8(BMW, BNT);
+            if (stall) gemm::wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook
+            int g = 0;
+            for (int i = 0; i < my_tiles && !*abort_v; ++i) {
+                const int ab = i & 1;
+                if (!gemm::wait_or_abort(&sm.accempty[ab], ((i >> 1) & 1) ^ 1, sm.abort, wait_limit)) break;
+                tc::tc_fence_after();
+                const uint32_t acc = tmem + ab * BNT;
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb, ++g) {
+                    const int s = g % STAGES, sa = g % ASTAGES;
+                    if (!gemm::wait_or_abort(&sm.full[s], (g / STAGES) & 1, sm.abort, wait_limit) ||
+                        !gemm::wait_or_abort(&sm.afull[sa], (g / ASTAGES) & 1, sm.abort, wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t x_addr = tc::smem_u32(sm.act + s * ACT_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)
+                        tc::mma_i8_ts(acc, tmem + A_COL + 32 * sa + 8 * k, tc::smem_desc_sw128(x_addr + 32 * k), idesc,
+                                      (kb > 0 || k > 0) ? 1u : 0u);
+                    tc::mma_commit(&sm.empty[s]);
+                    tc::mma_commit(&sm.aempty[sa]);
+                }
+                if (!ok) break;
+                tc::mma_commit(&sm.accfull[ab]);
+            }
+            tc::mma_commit(sm.done);  // every MMA issued, also after an abort
+        }
+    } else if (warp < 2 + kDecWarps) {
+        const int grp = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int first = (r >> 2) & 1;
+        const int total = my_tiles * num_kb;
+        for (int g = grp; g < total; g += kGroups) {  // ------------------------- decoders
+            const int s = g % STAGES, sa = g % ASTAGES;
+            bool ok = gemm::wait_or_abort(&sm.full[s], (g / STAGES) & 1, sm.abort, wait_limit) &&
+                      gemm::wait_or_abort(&sm.aempty[sa], ((g / ASTAGES) & 1) ^ 1, sm.abort, wait_limit);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc::tc_fence_after();
+            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 32;
+            const uint4 wa = *reinterpret_cast<const uint4*>(crow + 16 * first);
+            const uint4 wb = *reinterpret_cast<const uint4*>(crow + 16 * (first ^ 1));
+            const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t d[4];
+                decode_word_natural(words[c], lut, d);
+                v[4 * c] = d[0];
+                v[4 * c + 1] = d[1];
+                v[4 * c + 2] = d[2];
+                v[4 * c + 3] = d[3];
+            }
+            tc::tmem_st_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + 32 * sa, v);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.afull[sa]);
+        }
+    } else {
+        const int quarter = warp & 3;  // ------------------------------------------ epilogue
+        const int r = quarter * 32 + lane;
+        const int et = threadIdx.x - 32 * (2 + kDecWarps);  // 0..127
+        // Every epilogue warp runs every iteration (and both named barriers of it) even after an
+        // abort, so the barrier counts always match; `alive` only skips the work.
+        bool alive = true;
+        for (int i = 0; i < my_tiles; ++i) {
+            const int ab = i & 1;
+            const int tile = blockIdx.x + i * gridDim.x;
+            const int n0 = (tile % n_tiles_w) * BMW, t0 = (tile / n_tiles_w) * BNT;
+            {
+                const int t = t0 + et;
+                sm.sa[ab * BNT + et] = t < T ? s_a[t] : 0.0f;
+            }
+            epi_bar();
+            bool ok = alive && gemm::wait_or_abort(&sm.accfull[ab], (i >> 1) & 1, sm.abort, wait_limit) && !*abort_v;
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc::tc_fence_after();
+                const int n = n0 + r;
+                const float sw = n < N ? s_w[n] : 0.0f;
+#pragma unroll 1
+                for (int cc = 0; cc < BNT / 16; ++cc) {
+                    uint32_t acc[16];
+                    tc::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + ab * BNT + cc * 16, acc);
+                    tc::tmem_ld_wait();
+                    if (cc == BNT / 16 - 1) {  // every column of this accumulator is in registers
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&sm.accempty[ab]);
+                    }
+                    if (n < N) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int t = t0 + cc * 16 + j;
+                            if (t < T) {
+                                const float v =
+                                    __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[ab * BNT + cc * 16 + j]);
+                                gemm_ts::store_one<OutT>(y + (int64_t)t * N + n, v);
+                            }
+                        }
+                    }
+                }
+            } else {
+                alive = false;
+            }
+            epi_bar();  // sa[ab] is rewritten two tiles later, after every warp has used it
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        int zero = 0;
+        tc::mbar_wait_bounded(sm.done, 0, &zero, wait_limit);
+        __syncwarp();
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+static int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int v = 0;
+        cached[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0 ? v : 148;
+    }
+    return cached[dev];
+}
+
+template <typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    auto encode = gemm::get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap mx, mc;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {BK, BNT};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16) * 4};
+        const cuuint32_t box[2] = {BK / 16, BMW};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const cudaError_t e = ensure_smem(w2a4_gemm_tsp_kernel<OutT>, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = ((N + BMW - 1) / BMW) * ((T + BNT - 1) / BNT);
+    if (tiles > 0x7fffffff) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<int64_t>(tiles, num_sms());
+    const int stall = gemm::g_stall_next ? 1 : 0;
+    gemm::g_stall_next = false;
+    w2a4_gemm_tsp_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
+                                                                  gemm::g_wait_limit, stall);
+    return cudaGetLastError();
+}
+
+}  // namespace gemm_tsp
+
+cudaError_t launch_linear_gemm_tsp(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                                   int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (f16) return gemm_tsp::launch_t<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return gemm_tsp::launch_t<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
 
 cudaError_t launch_linear_gemm_ts(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
                                   int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
