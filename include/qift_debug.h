@@ -32,7 +32,8 @@ qift_status qift_debug_set_pdl(int32_t enable);
 /* Pin the kernel family qift_linear uses: 0 = automatic (by batch size), 1 = CUDA-core GEMV,
  * 2 = tensor-core skinny GEMM (tokens <= 16, n_in % 64 == 0), 3 = tcgen05 GEMM with the
  * decoded weights in shared memory, 4 = tcgen05 GEMM with the decoded weights in tensor memory,
- * 5 = its persistent form with two accumulators (3, 4 and 5: n_in % 64 == 0).  A pinned family that cannot take a call makes it return
+ * 5 = its persistent form with two accumulators, 6 = its CTA-pair form (two SMs per tile,
+ * tcgen05 cta_group::2); 3 to 6 need n_in % 64 == 0.  A pinned family that cannot take a call makes it return
  * QIFT_ERR_UNSUPPORTED.  All families give bit-identical results; tests use this to cover
  * each on the same inputs.  Process-wide. */
 qift_status qift_debug_set_linear_path(int32_t path);

@@ -192,7 +192,7 @@ def test_single_linear_256x512_end_to_end():
 
 
 # ------------------------------------------------------------- tensor-core GEMM (prefill)
-@pytest.mark.parametrize("path", ["gemm", "gemm_ts", "gemm_tsp"])
+@pytest.mark.parametrize("path", ["gemm", "gemm_ts", "gemm_tsp", "gemm_pair"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(17, 256, 64), (128, 256, 128), (129, 257, 192), (300, 600, 4096),
                                     (256, 40, 640), (2048, 512, 11008), (64, 1000, 4160), (513, 130, 1024)])
@@ -210,7 +210,7 @@ def test_linear_gemm_parity(path, name, T, N, K):
 
 
 # ------------------------------------------------------- every kernel family, same inputs
-@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm", "gemm_ts", "gemm_tsp"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm", "gemm_ts", "gemm_tsp", "gemm_pair"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(1, 300, 4096), (2, 129, 512), (7, 64, 1024), (9, 257, 14336), (16, 4096, 4096),
                                     (16, 130, 64), (5, 1000, 11008)])

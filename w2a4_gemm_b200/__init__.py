@@ -197,7 +197,7 @@ def qift_debug_stall_next_gemm() -> None:
     _check(lib().qift_debug_stall_next_gemm(), "qift_debug_stall_next_gemm")
 
 
-LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3, "gemm_ts": 4, "gemm_tsp": 5}
+LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3, "gemm_ts": 4, "gemm_tsp": 5, "gemm_pair": 6}
 
 
 def qift_debug_set_linear_path(path) -> None:

@@ -113,16 +113,20 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
     int path = qift::debug_linear_path();
     if (path == qift::kPathAuto) {
         if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
-            path = qift::kPathGemmTs;
+            path = qift::kPathGemmPair;
         else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
             path = qift::kPathSkinny;
         else
             path = qift::kPathGemv;
-    } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs || path == qift::kPathGemmTsp) &&
+    } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs || path == qift::kPathGemmTsp ||
+                 path == qift::kPathGemmPair) &&
                 !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
                (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))) {
         return QIFT_ERR_UNSUPPORTED;
     }
+    if (path == qift::kPathGemmPair)
+        return from_cuda(qift::launch_linear_gemm_pair(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
+                                                       n_in, y, f16, s));
     if (path == qift::kPathGemmTsp)
         return from_cuda(qift::launch_linear_gemm_tsp(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
                                                       n_in, y, f16, s));
@@ -172,7 +176,7 @@ qift_status qift_debug_set_wait_limit(int64_t cycles) {
 }
 
 qift_status qift_debug_set_linear_path(int32_t path) {
-    if (path < 0 || path > 5) return QIFT_ERR_INVALID_ARG;
+    if (path < 0 || path > 6) return QIFT_ERR_INVALID_ARG;
     qift::debug_set_linear_path(path);
     return QIFT_OK;
 }

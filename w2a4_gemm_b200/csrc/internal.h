@@ -51,7 +51,7 @@ cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t
                                cudaStream_t s);
 
 // Test hooks behind qift_debug.h.
-enum LinearPath { kPathAuto = 0, kPathGemv = 1, kPathSkinny = 2, kPathGemm = 3, kPathGemmTs = 4, kPathGemmTsp = 5 };
+enum LinearPath { kPathAuto = 0, kPathGemv = 1, kPathSkinny = 2, kPathGemm = 3, kPathGemmTs = 4, kPathGemmTsp = 5, kPathGemmPair = 6 };
 void debug_set_linear_path(int path);
 int debug_linear_path();
 void debug_set_pdl(bool on);
@@ -63,6 +63,10 @@ void debug_stall_next_gemm();
 cudaError_t launch_linear_gemm_ts(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                   int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                   cudaStream_t s);
+
+// Tensor-memory-A GEMM on CTA pairs (tcgen05 cta_group::2): the default prefill path.
+cudaError_t launch_linear_gemm_pair(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                    int set, int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s);
 
 // Persistent tensor-memory-A GEMM (double-buffered accumulators, overlapped epilogue).
 cudaError_t launch_linear_gemm_tsp(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,

@@ -898,6 +898,327 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 
 }  // namespace gemm_tsp
 
+// =====================================================================================
+// CTA-pair variant of the tensor-memory-A GEMM.  A cluster of two CTAs on two SMs computes a
+// 256-weight-row x 256-token tile with pair MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256):
+// each CTA decodes its own 128 weight rows into its own tensor memory and stages only its half
+// of the activation tile (128 tokens); the two tensor cores exchange the B halves on chip.  Per
+// SM this halves the activation bytes fetched per multiply-add relative to the single-CTA
+// kernel.
+//   warp 0        TMA producer of this CTA (8-stage ring: 128 tokens x 128 B + 128 x 32 B codes)
+//   warp 1        TMEM owner of this CTA; in rank 0 also the MMA issuer for the pair
+//   warps 2..17   decoders (four groups, K blocks round-robin), then the epilogue of this
+//                 CTA's 128 accumulator rows
+// One ring of STAGES slots covers both the shared-memory stages and the tensor-memory A stages,
+// so a single commit per K block (`consumed`, arriving in both CTAs) frees both.  Rank 0's
+// decoders also wait for the pair's activation halves (both CTAs' loads complete on rank 0's
+// `full`), so the decoders' `afull` (eight arrivals: four warps per CTA) is the only barrier the
+// MMA issuer waits on.  The single MMA-issuing thread is what paces the tensor core when its
+// loop carries more than one wait and one commit per K block, hence this layout.
+// =====================================================================================
+namespace gemm_pair {
+
+constexpr int BMW = 128;                          // weight rows per CTA (pair MMA M = 256)
+constexpr int BNT = 256;                          // tokens per pair tile (MMA N)
+constexpr int BNH = BNT / 2;                      // tokens of B staged by each CTA
+constexpr int BK = 128;
+constexpr int STAGES = 8;                         // shared-memory slots = tensor-memory A stages
+constexpr int kGroups = 4;
+constexpr int kDecWarps = 4 * kGroups;
+constexpr int kThreads = 64 + 32 * kDecWarps;
+constexpr int ACT_BYTES = BNH * BK;               // 16 KB
+constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 4 KB
+constexpr int BAR_BYTES = 512;
+constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + BAR_BYTES + BNT * 4;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t A_COL = 256;                   // A stage s at A_COL + 32 * s
+constexpr int STG_BYTES = 16 * 32 * 4;            // per-warp epilogue transpose buffer (fp32 worst case)
+static_assert(A_COL + 32 * STAGES <= TMEM_COLS, "tensor memory");
+static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier area");
+static_assert(kDecWarps * STG_BYTES <= STAGES * ACT_BYTES, "epilogue staging reuses the ring");
+static_assert((STAGES & (STAGES - 1)) == 0 && kGroups < STAGES, "stage arithmetic");
+static_assert(BK == 128, "the MMA loop issues four K = 32 steps per block");
+
+struct Smem {
+    uint8_t* act;
+    uint8_t* cod;
+    uint64_t* full;      // [STAGES] rank 0: both CTAs' activation halves landed
+    uint64_t* cfull;     // [STAGES] this CTA's codes landed
+    uint64_t* afull;     // [STAGES] rank 0: decoded weights of both CTAs in tensor memory
+    uint64_t* consumed;  // [STAGES] pair MMAs done with the slot and the A stage (both CTAs)
+    uint64_t* accum;
+    uint64_t* never;
+    uint32_t* tmem_base;
+    int* abort;
+    float* sa;           // [BNT] activation scales of the pair tile's tokens
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    Smem s;
+    s.act = base;
+    s.cod = s.act + STAGES * ACT_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.cod + STAGES * COD_BYTES);
+    s.full = bars;
+    s.cfull = s.full + STAGES;
+    s.afull = s.cfull + STAGES;
+    s.consumed = s.afull + STAGES;
+    s.accum = s.consumed + STAGES;
+    s.never = s.accum + 1;
+    s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
+    s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
+    s.sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + BAR_BYTES);
+    return s;
+}
+
+// One non-blocking probe, then the bounded wait (which records a timeout).
+__device__ __forceinline__ bool wait_fast(uint64_t* bar, uint32_t parity, int* abort, long long limit) {
+    return tc::mbar_try_wait(bar, parity) || gemm::wait_or_abort(bar, parity, abort, limit);
+}
+
+template <typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    w2a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
+                          const float* __restrict__ s_a, const float* __restrict__ s_w, uint32_t lut, int T, int N,
+                          int K, OutT* __restrict__ y, long long wait_limit, int stall) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = tc::cluster_ctarank();
+    const int n0 = (int)(blockIdx.x >> 1) * (2 * BMW) + (int)rank * BMW;  // this CTA's weight rows
+    const int t0 = blockIdx.y * BNT;                                        // the pair tile's tokens
+    const int tb = t0 + (int)rank * BNH;                                    // this CTA's B half
+    const int num_kb = (K + BK - 1) / BK;
+    // A box lying wholly outside the matrix is not fetched: its rows/tokens are never stored.
+    const bool has_act = tb < T, has_cod = n0 < N;
+    const uint32_t act_tx = (t0 + BNH < T ? 2u : 1u) * ACT_BYTES;  // rank 0: both halves' bytes
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&sm.full[s], 1);
+            tc::mbar_init(&sm.cfull[s], 1);
+            tc::mbar_init(&sm.afull[s], 8);  // four decoder warps in each CTA
+            tc::mbar_init(&sm.consumed[s], 1);
+        }
+        tc::mbar_init(sm.accum, 1);
+        tc::mbar_init(sm.never, 1);
+        *sm.abort = 0;
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&tmap_x);
+        tc::prefetch_tensormap(&tmap_c);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc_pair(sm.tmem_base, TMEM_COLS);
+        tc::tmem_relinquish_pair();
+    }
+    if (threadIdx.x >= 64 && threadIdx.x < 64 + BNT) {
+        const int t = t0 + threadIdx.x - 64;
+        sm.sa[threadIdx.x - 64] = t < T ? s_a[t] : 0.0f;
+    }
+    tc::tc_fence_before();
+    tc::cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or copy
+    tc::tc_fence_after();
+    const uint32_t tmem = *sm.tmem_base;
+    volatile int* abort_v = reinterpret_cast<volatile int*>(sm.abort);
+
+    if (warp == 0) {
+        if (lane == 0) {  // ------------------------------------------------ TMA producer
+            const uint32_t full0 = tc::cluster_addr(sm.full, 0);
+            int issued = 0;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
+                if (kb >= STAGES && !wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) break;
+                if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_tx);
+                tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
+                if (has_act) tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BK, tb);
+                if (has_cod) tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * (BK / 16), n0);
+                ++issued;
+            }
+            if (*abort_v) {
+                // Drain: the copies this thread started land before the CTA exits.  Rank 0 sees
+                // both halves of the activations on its own barriers; each CTA sees its codes.
+                int zero = 0;
+                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb) {
+                    const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
+                    if (rank == 0) tc::mbar_wait_bounded(&sm.full[s], ph, &zero, wait_limit);
+                    tc::mbar_wait_bounded(&sm.cfull[s], ph, &zero, wait_limit);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {  // -------------------------------------- pair MMA issuer
+            constexpr uint32_t idesc = tc::idesc_i8(2 * BMW, BNT);
+            const uint64_t desc0 = tc::smem_desc_sw128(tc::smem_u32(sm.act));
+            if (stall) gemm::wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook
+            // The wait for block kb + 1 sits between the MMAs of block kb, so it overlaps the
+            // MMAs already queued.
+            bool ok = !*abort_v && num_kb > 0 && wait_fast(&sm.afull[0], 0, sm.abort, wait_limit);
+            for (int kb = 0; ok && kb < num_kb; ++kb) {
+                const uint32_t s = kb & (STAGES - 1);
+                tc::tc_fence_after();
+                const uint64_t d = desc0 + (uint64_t)((s * ACT_BYTES) >> 4);
+                const uint32_t a = tmem + A_COL + 32 * s;
+                tc::mma_i8_ts_pair(tmem + ACC_COL, a, d, idesc, kb != 0 ? 1u : 0u);
+                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8, d + 2, idesc, 1u);
+                if (kb + 1 < num_kb)
+                    ok = wait_fast(&sm.afull[(kb + 1) & (STAGES - 1)], ((kb + 1) / STAGES) & 1, sm.abort, wait_limit);
+                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 16, d + 4, idesc, 1u);
+                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 24, d + 6, idesc, 1u);
+                tc::mma_commit_pair(&sm.consumed[s], 0x3);
+            }
+            if (*abort_v) {  // the peer must not store the tile either
+                tc::st_cluster_u32(sm.abort, 1, 1u);
+                asm volatile("fence.acq_rel.cluster;" ::: "memory");
+            }
+            tc::mma_commit_pair(sm.accum, 0x3);  // also after an abort, so both CTAs see the MMAs drained
+        }
+    } else {
+        const int grp = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int first = (r >> 2) & 1;
+        for (int kb = grp; kb < num_kb; kb += kGroups) {  // ---------------- decoders
+            const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
+            bool ok = wait_fast(&sm.cfull[s], ph, sm.abort, wait_limit) &&
+                      (kb < STAGES || wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) &&
+                      (rank != 0 || wait_fast(&sm.full[s], ph, sm.abort, wait_limit));
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc::tc_fence_after();
+            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 32;
+            const uint4 wa = *reinterpret_cast<const uint4*>(crow + 16 * first);
+            const uint4 wb = *reinterpret_cast<const uint4*>(crow + 16 * (first ^ 1));
+            const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
+            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t d[4];
+                decode_word_natural(words[c], lut, d);
+                v[4 * c] = d[0];
+                v[4 * c + 1] = d[1];
+                v[4 * c + 2] = d[2];
+                v[4 * c + 3] = d[3];
+            }
+            tc::tmem_st_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + 32 * s, v);
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive_cluster_relaxed(&sm.afull[s], 0);
+        }
+        // ---------------------------------------------------------------- epilogue
+        // Each warp owns 32 weight rows x 64 tokens.  Per 16-token chunk it scales the
+        // accumulators, transposes them through a private shared-memory buffer (the idle TMA
+        // ring) into [token][row] order and writes 16-byte pieces along n.
+        bool ok = gemm::wait_or_abort(sm.accum, 0, sm.abort, wait_limit) && !*abort_v;
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc::tc_fence_after();
+            const int n = n0 + r;
+            const float sw = n < N ? s_w[n] : 0.0f;
+            OutT* stg = reinterpret_cast<OutT*>(sm.act + (warp - 2) * STG_BYTES);
+            constexpr int EPP = 16 / sizeof(OutT);     // elements per 16-byte piece
+            constexpr int PPT = 32 / EPP;              // pieces per token row of the warp
+            const int nw = n0 + quarter * 32;          // first row of this warp
+            const bool vec_ok = ((int64_t)N * sizeof(OutT)) % 16 == 0;
+#pragma unroll 1
+            for (int cc = 0; cc < BNT / (16 * kGroups); ++cc) {
+                const int c0 = grp * (BNT / kGroups) + cc * 16;  // token column within the pair tile
+                uint32_t acc[16];
+                tc::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[c0 + j]);
+                    gemm_ts::store_one<OutT>(stg + j * 32 + lane, v);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < (16 * PPT) / 32; ++i) {
+                    const int p = lane + 32 * i;
+                    const int j = p / PPT, sub = p % PPT;
+                    const int t = t0 + c0 + j, nn = nw + sub * EPP;
+                    if (t < T) {
+                        OutT* dst = y + (int64_t)t * N + nn;
+                        const OutT* src = stg + j * 32 + sub * EPP;
+                        if (vec_ok && nn + EPP <= N) {
+                            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                        } else {
+                            for (int e = 0; e < EPP; ++e)
+                                if (nn + e < N) dst[e] = src[e];
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        // The pair MMAs read this CTA's shared and tensor memory: wait for the last of them.
+        int zero = 0;
+        tc::mbar_wait_bounded(sm.accum, 0, &zero, wait_limit);
+        __syncwarp();
+    }
+    // Neither CTA leaves (or frees its tensor memory) while the other may still read its
+    // memory or arrive on its barriers.
+    tc::cluster_sync();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc_pair(tmem, TMEM_COLS);
+    }
+}
+
+template <typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    auto encode = gemm::get_encode();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap mx, mc;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {BK, BNH};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 16), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 16) * 4};
+        const cuuint32_t box[2] = {BK / 16, BMW};
+        const cuuint32_t es[2] = {1, 1};
+        if (encode(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const cudaError_t e = ensure_smem(w2a4_gemm_pair_kernel<OutT>, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int64_t pairs = (N + 2 * BMW - 1) / (2 * BMW);
+    if (2 * pairs > 0x7fffffff) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)(2 * pairs), (unsigned)((T + BNT - 1) / BNT));
+    const int stall = gemm::g_stall_next ? 1 : 0;
+    gemm::g_stall_next = false;
+    w2a4_gemm_pair_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
+                                                                   gemm::g_wait_limit, stall);
+    return cudaGetLastError();
+}
+
+}  // namespace gemm_pair
+
+cudaError_t launch_linear_gemm_pair(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
+                                    int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
+    if (T == 0 || N == 0) return cudaSuccess;
+    const uint32_t lut = level_lut(set);
+    if (f16) return gemm_pair::launch_t<__half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return gemm_pair::launch_t<float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+}
+
 cudaError_t launch_linear_gemm_tsp(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
                                    int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
     if (T == 0 || N == 0) return cudaSuccess;
