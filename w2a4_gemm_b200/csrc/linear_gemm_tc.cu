@@ -905,7 +905,7 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 // of the activation tile (128 tokens); the two tensor cores exchange the B halves on chip.  Per
 // SM this halves the activation bytes fetched per multiply-add relative to the single-CTA
 // kernel.
-//   warp 0        TMA producer of this CTA (8-stage ring: 128 tokens x 128 B + 128 x 32 B codes)
+//   warp 0        TMA producer of this CTA (4-stage ring: 128 tokens x 256 B + 128 x 64 B codes)
 //   warp 1        TMEM owner of this CTA; in rank 0 also the MMA issuer for the pair
 //   warps 2..17   decoders (four groups, K blocks round-robin), then the epilogue of this
 //                 CTA's 128 accumulator rows
@@ -921,24 +921,25 @@ namespace gemm_pair {
 constexpr int BMW = 128;                          // weight rows per CTA (pair MMA M = 256)
 constexpr int BNT = 256;                          // tokens per pair tile (MMA N)
 constexpr int BNH = BNT / 2;                      // tokens of B staged by each CTA
-constexpr int BK = 128;
-constexpr int STAGES = 8;                         // shared-memory slots = tensor-memory A stages
+constexpr int BK = 256;                           // K bytes per block: two 128-byte swizzled columns
+constexpr int STAGES = 4;                         // shared-memory slots = tensor-memory A stages
 constexpr int kGroups = 4;
 constexpr int kDecWarps = 4 * kGroups;
 constexpr int kThreads = 64 + 32 * kDecWarps;
-constexpr int ACT_BYTES = BNH * BK;               // 16 KB
-constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 4 KB
+constexpr int ACT_HALF = BNH * 128;               // one 128-byte column of the activation block: 16 KB
+constexpr int ACT_BYTES = BNH * BK;               // 32 KB
+constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 8 KB (64-byte rows, 64-byte swizzle)
 constexpr int BAR_BYTES = 512;
 constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + BAR_BYTES + BNT * 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t A_COL = 256;                   // A stage s at A_COL + 32 * s
+constexpr uint32_t A_COL = 256;                   // A stage s at A_COL + 64 * s (BK / 4 columns)
 constexpr int STG_BYTES = 16 * 32 * 4;            // per-warp epilogue transpose buffer (fp32 worst case)
-static_assert(A_COL + 32 * STAGES <= TMEM_COLS, "tensor memory");
+static_assert(A_COL + (BK / 4) * STAGES <= TMEM_COLS, "tensor memory");
 static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier area");
 static_assert(kDecWarps * STG_BYTES <= STAGES * ACT_BYTES, "epilogue staging reuses the ring");
-static_assert((STAGES & (STAGES - 1)) == 0 && kGroups < STAGES, "stage arithmetic");
-static_assert(BK == 128, "the MMA loop issues four K = 32 steps per block");
+static_assert((STAGES & (STAGES - 1)) == 0 && kGroups <= STAGES, "stage arithmetic");
+static_assert(BK == 256, "the MMA loop issues eight K = 32 steps per block");
 
 struct Smem {
     uint8_t* act;
@@ -992,7 +993,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int num_kb = (K + BK - 1) / BK;
     // A box lying wholly outside the matrix is not fetched: its rows/tokens are never stored.
     const bool has_act = tb < T, has_cod = n0 < N;
-    const uint32_t act_tx = (t0 + BNH < T ? 2u : 1u) * ACT_BYTES;  // rank 0: both halves' bytes
+    // Rank 0 expects the activation bytes of both CTAs; the second 128-byte column of the last
+    // block is neither fetched nor multiplied when it lies wholly past K.
+    const uint32_t act_ctas = t0 + BNH < T ? 2u : 1u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1029,9 +1032,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int kb = 0; kb < num_kb; ++kb) {
                 const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
                 if (kb >= STAGES && !wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) break;
-                if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_tx);
+                const bool second = kb * BK + 128 < K;
+                if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_ctas * (second ? 2u : 1u) * ACT_HALF);
                 tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
-                if (has_act) tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BK, tb);
+                if (has_act) {
+                    tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BK, tb);
+                    if (second)
+                        tc::tma_load_2d_pair(sm.act + s * ACT_BYTES + ACT_HALF, &tmap_x, full0 + 8 * s, kb * BK + 128, tb);
+                }
                 if (has_cod) tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * (BK / 16), n0);
                 ++issued;
             }
@@ -1058,13 +1066,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t s = kb & (STAGES - 1);
                 tc::tc_fence_after();
                 const uint64_t d = desc0 + (uint64_t)((s * ACT_BYTES) >> 4);
-                const uint32_t a = tmem + A_COL + 32 * s;
+                const uint64_t d2 = d + (uint64_t)(ACT_HALF >> 4);
+                const uint32_t a = tmem + A_COL + (BK / 4) * s;
                 tc::mma_i8_ts_pair(tmem + ACC_COL, a, d, idesc, kb != 0 ? 1u : 0u);
-                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8, d + 2, idesc, 1u);
+#pragma unroll
+                for (int k = 1; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8 * k, d + 2 * k, idesc, 1u);
                 if (kb + 1 < num_kb)
                     ok = wait_fast(&sm.afull[(kb + 1) & (STAGES - 1)], ((kb + 1) / STAGES) & 1, sm.abort, wait_limit);
-                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 16, d + 4, idesc, 1u);
-                tc::mma_i8_ts_pair(tmem + ACC_COL, a + 24, d + 6, idesc, 1u);
+                if (kb * BK + 128 < K) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 32 + 8 * k, d2 + 2 * k, idesc, 1u);
+                }
                 tc::mma_commit_pair(&sm.consumed[s], 0x3);
             }
             if (*abort_v) {  // the peer must not store the tile either
@@ -1077,7 +1089,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int grp = (warp - 2) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
-        const int first = (r >> 2) & 1;
+        const int swz = (r >> 1) & 3;  // 64-byte TMA swizzle: chunk c of row r sits at c ^ swz
         for (int kb = grp; kb < num_kb; kb += kGroups) {  // ---------------- decoders
             const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
             bool ok = wait_fast(&sm.cfull[s], ph, sm.abort, wait_limit) &&
@@ -1085,22 +1097,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       (rank != 0 || wait_fast(&sm.full[s], ph, sm.abort, wait_limit));
             if (!__all_sync(0xffffffffu, ok)) break;
             tc::tc_fence_after();
-            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 32;
-            const uint4 wa = *reinterpret_cast<const uint4*>(crow + 16 * first);
-            const uint4 wb = *reinterpret_cast<const uint4*>(crow + 16 * (first ^ 1));
-            const uint4 w0 = first ? wb : wa, w1 = first ? wa : wb;
-            const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint32_t v[32];
+            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 64;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + (BK / 4) * s;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t d[4];
-                decode_word_natural(words[c], lut, d);
-                v[4 * c] = d[0];
-                v[4 * c + 1] = d[1];
-                v[4 * c + 2] = d[2];
-                v[4 * c + 3] = d[3];
+            for (int h = 0; h < 2; ++h) {  // 128 K bytes (eight code words) per tensor-memory store
+                const uint4 w0 = *reinterpret_cast<const uint4*>(crow + 16 * ((2 * h) ^ swz));
+                const uint4 w1 = *reinterpret_cast<const uint4*>(crow + 16 * ((2 * h + 1) ^ swz));
+                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t d[4];
+                    decode_word_natural(words[c], lut, d);
+                    v[4 * c] = d[0];
+                    v[4 * c + 1] = d[1];
+                    v[4 * c + 2] = d[2];
+                    v[4 * c + 3] = d[3];
+                }
+                tc::tmem_st_32x32b_x32(taddr + 32 * h, v);
             }
-            tc::tmem_st_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + 32 * s, v);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             __syncwarp();
@@ -1180,7 +1195,7 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     {
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)K};
-        const cuuint32_t box[2] = {BK, BNH};
+        const cuuint32_t box[2] = {128, BNH};
         const cuuint32_t es[2] = {1, 1};
         if (encode(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(q), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1193,7 +1208,7 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
         const cuuint32_t box[2] = {BK / 16, BMW};
         const cuuint32_t es[2] = {1, 1};
         if (encode(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
