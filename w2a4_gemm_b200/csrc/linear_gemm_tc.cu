@@ -899,22 +899,24 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
 }  // namespace gemm_tsp
 
 // =====================================================================================
-// CTA-pair variant of the tensor-memory-A GEMM.  A cluster of two CTAs on two SMs computes a
-// 256-weight-row x 256-token tile with pair MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256):
-// each CTA decodes its own 128 weight rows into its own tensor memory and stages only its half
-// of the activation tile (128 tokens); the two tensor cores exchange the B halves on chip.  Per
-// SM this halves the activation bytes fetched per multiply-add relative to the single-CTA
-// kernel.
-//   warp 0        TMA producer of this CTA (4-stage ring: 128 tokens x 256 B + 128 x 64 B codes)
-//   warp 1        TMEM owner of this CTA; in rank 0 also the MMA issuer for the pair
-//   warps 2..17   decoders (four groups, K blocks round-robin), then the epilogue of this
-//                 CTA's 128 accumulator rows
+// CTA-pair GEMM, persistent.  A cluster of two CTAs on two SMs computes 256-weight-row x
+// 256-token tiles with pair MMAs (tcgen05.mma.cta_group::2, M = 256, N = 256): each CTA decodes
+// its own 128 weight rows into its own tensor memory and stages only its half of the activation
+// tile (128 tokens); the two tensor cores exchange the B halves on chip, which halves the
+// activation bytes each SM fetches per multiply-add.  Each cluster walks a list of tiles; the
+// TMA ring and the decoders run straight on from one tile into the next, and dedicated epilogue
+// warps drain the accumulator into shared memory, release it to the next tile's MMAs and write
+// the tile out while those run, so per-tile start-up and write-out are hidden.
+//   warp 0          TMA producer of this CTA (4-stage ring: 128 tokens x 256 B + 128 x 64 B codes)
+//   warp 1          TMEM owner of this CTA; in rank 0 also the MMA issuer for the pair
+//   warps 2..9      decoders: group g (4 warps) fills ring stages g and g + 2
+//   warps 10..25    epilogue: four warps per TMEM lane quarter, a quarter of the columns each
 // One ring of STAGES slots covers both the shared-memory stages and the tensor-memory A stages,
 // so a single commit per K block (`consumed`, arriving in both CTAs) frees both.  Rank 0's
 // decoders also wait for the pair's activation halves (both CTAs' loads complete on rank 0's
 // `full`), so the decoders' `afull` (eight arrivals: four warps per CTA) is the only barrier the
-// MMA issuer waits on.  The single MMA-issuing thread is what paces the tensor core when its
-// loop carries more than one wait and one commit per K block, hence this layout.
+// MMA issuer waits on inside a tile; the single MMA-issuing thread otherwise paces the tensor
+// core with its own instruction latency.
 // =====================================================================================
 namespace gemm_pair {
 
@@ -923,36 +925,43 @@ constexpr int BNT = 256;                          // tokens per pair tile (MMA N
 constexpr int BNH = BNT / 2;                      // tokens of B staged by each CTA
 constexpr int BK = 256;                           // K bytes per block: two 128-byte swizzled columns
 constexpr int STAGES = 4;                         // shared-memory slots = tensor-memory A stages
-constexpr int kGroups = 4;
+constexpr int kGroups = 2;
 constexpr int kDecWarps = 4 * kGroups;
-constexpr int kThreads = 64 + 32 * kDecWarps;
+constexpr int kEpiWarps = 16;
+constexpr int kEpiBase = 2 + kDecWarps;           // first epilogue warp
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 32 * (kEpiBase + kEpiWarps);
 constexpr int ACT_HALF = BNH * 128;               // one 128-byte column of the activation block: 16 KB
 constexpr int ACT_BYTES = BNH * BK;               // 32 KB
 constexpr int COD_BYTES = BMW * (BK / 16) * 4;    // 8 KB (64-byte rows, 64-byte swizzle)
-constexpr int BAR_BYTES = 512;
-constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + 1024 + BAR_BYTES + BNT * 4;
+constexpr int STG_BYTES = 64 * 1024;              // epilogue staging: [columns of a pass][128 rows]
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * (ACT_BYTES + COD_BYTES) + STG_BYTES + 1024 + BAR_BYTES + BNT * 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
 constexpr uint32_t A_COL = 256;                   // A stage s at A_COL + 64 * s (BK / 4 columns)
-constexpr int STG_BYTES = 16 * 32 * 4;            // per-warp epilogue transpose buffer (fp32 worst case)
 static_assert(A_COL + (BK / 4) * STAGES <= TMEM_COLS, "tensor memory");
-static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier area");
-static_assert(kDecWarps * STG_BYTES <= STAGES * ACT_BYTES, "epilogue staging reuses the ring");
-static_assert((STAGES & (STAGES - 1)) == 0 && kGroups <= STAGES, "stage arithmetic");
+static_assert((4 * STAGES + 4) * 8 + 8 <= BAR_BYTES, "barrier area");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(STAGES % kGroups == 0, "decoder group g fills ring stages g, g + kGroups, ...");
 static_assert(BK == 256, "the MMA loop issues eight K = 32 steps per block");
+static_assert(kEpiThreads >= BNT, "one epilogue thread per token scale");
 
 struct Smem {
     uint8_t* act;
     uint8_t* cod;
+    uint8_t* stg;
     uint64_t* full;      // [STAGES] rank 0: both CTAs' activation halves landed
     uint64_t* cfull;     // [STAGES] this CTA's codes landed
     uint64_t* afull;     // [STAGES] rank 0: decoded weights of both CTAs in tensor memory
     uint64_t* consumed;  // [STAGES] pair MMAs done with the slot and the A stage (both CTAs)
-    uint64_t* accum;
+    uint64_t* accfull;   // the tile's MMAs are complete (both CTAs)
+    uint64_t* accfree;   // rank 0: both CTAs' epilogues have read the accumulator
+    uint64_t* done;      // every MMA issued has completed (both CTAs)
     uint64_t* never;
     uint32_t* tmem_base;
     int* abort;
-    float* sa;           // [BNT] activation scales of the pair tile's tokens
+    float* sa;           // [BNT] activation scales of the tile being written out
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
@@ -960,13 +969,16 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
     Smem s;
     s.act = base;
     s.cod = s.act + STAGES * ACT_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s.cod + STAGES * COD_BYTES);
+    s.stg = s.cod + STAGES * COD_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s.stg + STG_BYTES);
     s.full = bars;
     s.cfull = s.full + STAGES;
     s.afull = s.cfull + STAGES;
     s.consumed = s.afull + STAGES;
-    s.accum = s.consumed + STAGES;
-    s.never = s.accum + 1;
+    s.accfull = s.consumed + STAGES;
+    s.accfree = s.accfull + 1;
+    s.done = s.accfree + 1;
+    s.never = s.done + 1;
     s.tmem_base = reinterpret_cast<uint32_t*>(s.never + 1);
     s.abort = reinterpret_cast<int*>(s.tmem_base + 1);
     s.sa = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + BAR_BYTES);
@@ -978,6 +990,21 @@ __device__ __forceinline__ bool wait_fast(uint64_t* bar, uint32_t parity, int* a
     return tc::mbar_try_wait(bar, parity) || gemm::wait_or_abort(bar, parity, abort, limit);
 }
 
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory"); }
+
+struct Tile {
+    int n0;  // this CTA's first weight row
+    int t0;  // the pair tile's first token
+};
+
+__device__ __forceinline__ Tile tile_of(int i, int pairs_x, uint32_t rank) {
+    const int tile = (int)(blockIdx.x >> 1) + i * (int)(gridDim.x >> 1);
+    Tile t;
+    t.n0 = (tile % pairs_x) * (2 * BMW) + (int)rank * BMW;
+    t.t0 = (tile / pairs_x) * BNT;
+    return t;
+}
+
 template <typename OutT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     w2a4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_c,
@@ -987,15 +1014,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const Smem sm = carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = tc::cluster_ctarank();
-    const int n0 = (int)(blockIdx.x >> 1) * (2 * BMW) + (int)rank * BMW;  // this CTA's weight rows
-    const int t0 = blockIdx.y * BNT;                                        // the pair tile's tokens
-    const int tb = t0 + (int)rank * BNH;                                    // this CTA's B half
+    const int pairs_x = (N + 2 * BMW - 1) / (2 * BMW);
+    const int tiles = pairs_x * ((T + BNT - 1) / BNT);
+    const int cl = (int)(blockIdx.x >> 1), clusters = (int)(gridDim.x >> 1);
+    const int my_tiles = cl < tiles ? (tiles - 1 - cl) / clusters + 1 : 0;
     const int num_kb = (K + BK - 1) / BK;
-    // A box lying wholly outside the matrix is not fetched: its rows/tokens are never stored.
-    const bool has_act = tb < T, has_cod = n0 < N;
-    // Rank 0 expects the activation bytes of both CTAs; the second 128-byte column of the last
-    // block is neither fetched nor multiplied when it lies wholly past K.
-    const uint32_t act_ctas = t0 + BNH < T ? 2u : 1u;
+    const int total = my_tiles * num_kb;  // K blocks this cluster streams through the ring
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1004,7 +1028,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc::mbar_init(&sm.afull[s], 8);  // four decoder warps in each CTA
             tc::mbar_init(&sm.consumed[s], 1);
         }
-        tc::mbar_init(sm.accum, 1);
+        tc::mbar_init(sm.accfull, 1);
+        tc::mbar_init(sm.accfree, 2 * kEpiWarps);
+        tc::mbar_init(sm.done, 1);
         tc::mbar_init(sm.never, 1);
         *sm.abort = 0;
         tc::fence_mbar_init();
@@ -1015,10 +1041,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc::tmem_alloc_pair(sm.tmem_base, TMEM_COLS);
         tc::tmem_relinquish_pair();
     }
-    if (threadIdx.x >= 64 && threadIdx.x < 64 + BNT) {
-        const int t = t0 + threadIdx.x - 64;
-        sm.sa[threadIdx.x - 64] = t < T ? s_a[t] : 0.0f;
-    }
     tc::tc_fence_before();
     tc::cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or copy
     tc::tc_fence_after();
@@ -1028,27 +1050,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {  // ------------------------------------------------ TMA producer
             const uint32_t full0 = tc::cluster_addr(sm.full, 0);
-            int issued = 0;
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
-                if (kb >= STAGES && !wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) break;
-                const bool second = kb * BK + 128 < K;
-                if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_ctas * (second ? 2u : 1u) * ACT_HALF);
-                tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
-                if (has_act) {
-                    tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BK, tb);
-                    if (second)
-                        tc::tma_load_2d_pair(sm.act + s * ACT_BYTES + ACT_HALF, &tmap_x, full0 + 8 * s, kb * BK + 128, tb);
+            int g = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < my_tiles; ++i) {
+                const Tile tl = tile_of(i, pairs_x, rank);
+                const int tb = tl.t0 + (int)rank * BNH;  // this CTA's B half
+                // A box lying wholly outside the matrix is not fetched: its rows/tokens are never
+                // stored.  Rank 0 expects the activation bytes of both CTAs; the second 128-byte
+                // column of the last block is neither fetched nor multiplied when wholly past K.
+                const bool has_act = tb < T, has_cod = tl.n0 < N;
+                const uint32_t act_ctas = tl.t0 + BNH < T ? 2u : 1u;
+                for (int kb = 0; kb < num_kb; ++kb, ++g) {
+                    const uint32_t s = g & (STAGES - 1), ph = (g / STAGES) & 1;
+                    if (g >= STAGES && !wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) {
+                        ok = false;
+                        break;
+                    }
+                    const bool second = kb * BK + 128 < K;
+                    if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_ctas * (second ? 2u : 1u) * ACT_HALF);
+                    tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
+                    if (has_act) {
+                        tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BK, tb);
+                        if (second)
+                            tc::tma_load_2d_pair(sm.act + s * ACT_BYTES + ACT_HALF, &tmap_x, full0 + 8 * s,
+                                                 kb * BK + 128, tb);
+                    }
+                    if (has_cod)
+                        tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * (BK / 16), tl.n0);
                 }
-                if (has_cod) tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * (BK / 16), n0);
-                ++issued;
             }
             if (*abort_v) {
                 // Drain: the copies this thread started land before the CTA exits.  Rank 0 sees
                 // both halves of the activations on its own barriers; each CTA sees its codes.
                 int zero = 0;
-                for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb) {
-                    const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
+                for (int q = g > STAGES ? g - STAGES : 0; q < g; ++q) {
+                    const uint32_t s = q & (STAGES - 1), ph = (q / STAGES) & 1;
                     if (rank == 0) tc::mbar_wait_bounded(&sm.full[s], ph, &zero, wait_limit);
                     tc::mbar_wait_bounded(&sm.cfull[s], ph, &zero, wait_limit);
                 }
@@ -1059,46 +1095,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             constexpr uint32_t idesc = tc::idesc_i8(2 * BMW, BNT);
             const uint64_t desc0 = tc::smem_desc_sw128(tc::smem_u32(sm.act));
             if (stall) gemm::wait_or_abort(sm.never, 0, sm.abort, wait_limit);  // test hook
-            // The wait for block kb + 1 sits between the MMAs of block kb, so it overlaps the
-            // MMAs already queued.
-            bool ok = !*abort_v && num_kb > 0 && wait_fast(&sm.afull[0], 0, sm.abort, wait_limit);
-            for (int kb = 0; ok && kb < num_kb; ++kb) {
-                const uint32_t s = kb & (STAGES - 1);
-                tc::tc_fence_after();
-                const uint64_t d = desc0 + (uint64_t)((s * ACT_BYTES) >> 4);
-                const uint64_t d2 = d + (uint64_t)(ACT_HALF >> 4);
-                const uint32_t a = tmem + A_COL + (BK / 4) * s;
-                tc::mma_i8_ts_pair(tmem + ACC_COL, a, d, idesc, kb != 0 ? 1u : 0u);
+            // The wait for block g + 1 sits between the MMAs of block g, so it overlaps the MMAs
+            // already queued; a tile's first MMA also waits until the epilogue has drained the
+            // previous tile's accumulator.
+            bool ok = !*abort_v && (total == 0 || wait_fast(&sm.afull[0], 0, sm.abort, wait_limit));
+            int g = 0;
+            for (int i = 0; ok && i < my_tiles; ++i) {
+                if (i > 0 && !wait_fast(sm.accfree, (i - 1) & 1, sm.abort, wait_limit)) break;
+                for (int kb = 0; kb < num_kb; ++kb, ++g) {
+                    const uint32_t s = g & (STAGES - 1);
+                    tc::tc_fence_after();
+                    const uint64_t d = desc0 + (uint64_t)((s * ACT_BYTES) >> 4);
+                    const uint64_t d2 = d + (uint64_t)(ACT_HALF >> 4);
+                    const uint32_t a = tmem + A_COL + (BK / 4) * s;
+                    tc::mma_i8_ts_pair(tmem + ACC_COL, a, d, idesc, kb != 0 ? 1u : 0u);
 #pragma unroll
-                for (int k = 1; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8 * k, d + 2 * k, idesc, 1u);
-                if (kb + 1 < num_kb)
-                    ok = wait_fast(&sm.afull[(kb + 1) & (STAGES - 1)], ((kb + 1) / STAGES) & 1, sm.abort, wait_limit);
-                if (kb * BK + 128 < K) {
+                    for (int k = 1; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8 * k, d + 2 * k, idesc, 1u);
+                    if (g + 1 < total)
+                        ok = wait_fast(&sm.afull[(g + 1) & (STAGES - 1)], ((g + 1) / STAGES) & 1, sm.abort, wait_limit);
+                    if (kb * BK + 128 < K) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 32 + 8 * k, d2 + 2 * k, idesc, 1u);
+                        for (int k = 0; k < 4; ++k)
+                            tc::mma_i8_ts_pair(tmem + ACC_COL, a + 32 + 8 * k, d2 + 2 * k, idesc, 1u);
+                    }
+                    tc::mma_commit_pair(&sm.consumed[s], 0x3);
+                    if (!ok) break;
                 }
-                tc::mma_commit_pair(&sm.consumed[s], 0x3);
+                if (!ok) break;
+                tc::mma_commit_pair(sm.accfull, 0x3);
             }
-            if (*abort_v) {  // the peer must not store the tile either
+            if (*abort_v) {  // the peer must not store its tiles either
                 tc::st_cluster_u32(sm.abort, 1, 1u);
                 asm volatile("fence.acq_rel.cluster;" ::: "memory");
             }
-            tc::mma_commit_pair(sm.accum, 0x3);  // also after an abort, so both CTAs see the MMAs drained
+            tc::mma_commit_pair(sm.done, 0x3);  // also after an abort, so both CTAs see the MMAs drained
         }
-    } else {
-        const int grp = (warp - 2) >> 2;
+    } else if (warp < kEpiBase) {
+        const int grp = (warp - 2) >> 2;  // fills ring stages grp, grp + kGroups, ...
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const int swz = (r >> 1) & 3;  // 64-byte TMA swizzle: chunk c of row r sits at c ^ swz
-        for (int kb = grp; kb < num_kb; kb += kGroups) {  // ---------------- decoders
-            const uint32_t s = kb & (STAGES - 1), ph = (kb / STAGES) & 1;
+        for (int g = grp; g < total; g += kGroups) {  // ---------------------- decoders
+            const uint32_t s = g & (STAGES - 1), ph = (g / STAGES) & 1;
             bool ok = wait_fast(&sm.cfull[s], ph, sm.abort, wait_limit) &&
-                      (kb < STAGES || wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) &&
+                      (g < STAGES || wait_fast(&sm.consumed[s], ph ^ 1, sm.abort, wait_limit)) &&
                       (rank != 0 || wait_fast(&sm.full[s], ph, sm.abort, wait_limit));
             if (!__all_sync(0xffffffffu, ok)) break;
-            tc::tc_fence_after();
-            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 64;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + (BK / 4) * s;
+            const uint8_t* crow = sm.cod + s * COD_BYTES + r * 64;
+            tc::tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // 128 K bytes (eight code words) per tensor-memory store
                 const uint4 w0 = *reinterpret_cast<const uint4*>(crow + 16 * ((2 * h) ^ swz));
@@ -1121,50 +1166,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive_cluster_relaxed(&sm.afull[s], 0);
         }
+    } else {
         // ---------------------------------------------------------------- epilogue
-        // Each warp owns 32 weight rows x 64 tokens.  Per 16-token chunk it scales the
-        // accumulators, transposes them through a private shared-memory buffer (the idle TMA
-        // ring) into [token][row] order and writes 16-byte pieces along n.
-        bool ok = gemm::wait_or_abort(sm.accum, 0, sm.abort, wait_limit) && !*abort_v;
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-            tc::tc_fence_after();
-            const int n = n0 + r;
-            const float sw = n < N ? s_w[n] : 0.0f;
-            OutT* stg = reinterpret_cast<OutT*>(sm.act + (warp - 2) * STG_BYTES);
-            constexpr int EPP = 16 / sizeof(OutT);     // elements per 16-byte piece
-            constexpr int PPT = 32 / EPP;              // pieces per token row of the warp
-            const int nw = n0 + quarter * 32;          // first row of this warp
-            const bool vec_ok = ((int64_t)N * sizeof(OutT)) % 16 == 0;
+        // Warp (quarter, column group): 32 weight rows, a quarter of each pass's columns.  Per tile:
+        // drain the accumulator (scaled, converted) into the staging buffer in [token][row]
+        // order -- in two passes of 128 columns for fp32 output -- release the accumulator after
+        // the last pass's reads, then write 16-byte pieces along n.  Every epilogue warp runs
+        // every named barrier of every tile, also after an abort (`alive` only skips the work).
+        constexpr int CPP = STG_BYTES / (BMW * (int)sizeof(OutT));  // columns per pass: 256 / 128
+        constexpr int PASSES = BNT / CPP;
+        constexpr int EPP = 16 / sizeof(OutT);                      // elements per 16-byte piece
+        constexpr int PPR = BMW / EPP;                              // pieces per token row
+        constexpr int CPW = CPP / 4;                                // columns per warp per pass
+        const int et = threadIdx.x - 32 * kEpiBase;                 // 0 .. kEpiThreads - 1
+        const int quarter = warp & 3, cgrp = (warp - kEpiBase) >> 2;
+        const int r = quarter * 32 + lane;
+        OutT* stg = reinterpret_cast<OutT*>(sm.stg);
+        const bool vec_ok = ((int64_t)N * sizeof(OutT)) % 16 == 0;
+        bool alive = true;
+        for (int i = 0; i < my_tiles; ++i) {
+            const Tile tl = tile_of(i, pairs_x, rank);
+            if (et < BNT) sm.sa[et] = tl.t0 + et < T ? s_a[tl.t0 + et] : 0.0f;
+            const float sw = tl.n0 + r < N ? s_w[tl.n0 + r] : 0.0f;
+            epi_bar();  // token scales in place
+            bool ok = alive && wait_fast(sm.accfull, i & 1, sm.abort, wait_limit) && !*abort_v;
+            alive = __all_sync(0xffffffffu, ok);
+            for (int p = 0; p < PASSES; ++p) {
+                if (alive) {
+                    tc::tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < BNT / (16 * kGroups); ++cc) {
-                const int c0 = grp * (BNT / kGroups) + cc * 16;  // token column within the pair tile
-                uint32_t acc[16];
-                tc::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
-                tc::tmem_ld_wait();
+                    for (int cc = 0; cc < CPW / 32; ++cc) {
+                        const int cl0 = cgrp * CPW + cc * 32;  // column within the pass
+                        const int c0 = p * CPP + cl0;         // column within the tile
+                        uint32_t acc[32];
+                        tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
+                        tc::tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[c0 + j]);
-                    gemm_ts::store_one<OutT>(stg + j * 32 + lane, v);
+                        for (int j = 0; j < 32; ++j) {
+                            const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[c0 + j]);
+                            gemm_ts::store_one<OutT>(stg + (cl0 + j) * BMW + r, v);
+                        }
+                    }
+                    if (p == PASSES - 1) {  // every column of the accumulator has been read
+                        tc::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive_cluster_relaxed(sm.accfree, 0);
+                    }
                 }
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < (16 * PPT) / 32; ++i) {
-                    const int p = lane + 32 * i;
-                    const int j = p / PPT, sub = p % PPT;
-                    const int t = t0 + c0 + j, nn = nw + sub * EPP;
-                    if (t < T) {
-                        OutT* dst = y + (int64_t)t * N + nn;
-                        const OutT* src = stg + j * 32 + sub * EPP;
-                        if (vec_ok && nn + EPP <= N) {
-                            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-                        } else {
-                            for (int e = 0; e < EPP; ++e)
-                                if (nn + e < N) dst[e] = src[e];
+                epi_bar();  // staging complete
+                if (alive) {
+#pragma unroll 2
+                    for (int q = et; q < CPP * PPR; q += kEpiThreads) {
+                        const int j = q / PPR, sub = q % PPR;
+                        const int t = tl.t0 + p * CPP + j, nn = tl.n0 + sub * EPP;
+                        if (t < T) {
+                            OutT* dst = y + (int64_t)t * N + nn;
+                            const OutT* src = stg + j * BMW + sub * EPP;
+                            if (vec_ok && nn + EPP <= N) {
+                                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                            } else {
+                                for (int e = 0; e < EPP; ++e)
+                                    if (nn + e < N) dst[e] = src[e];
+                            }
                         }
                     }
                 }
-                __syncwarp();
+                epi_bar();  // staging free again
             }
         }
     }
@@ -1174,7 +1241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         // The pair MMAs read this CTA's shared and tensor memory: wait for the last of them.
         int zero = 0;
-        tc::mbar_wait_bounded(sm.accum, 0, &zero, wait_limit);
+        tc::mbar_wait_bounded(sm.done, 0, &zero, wait_limit);
         __syncwarp();
     }
     // Neither CTA leaves (or frees its tensor memory) while the other may still read its
@@ -1184,6 +1251,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         tc::tmem_dealloc_pair(tmem, TMEM_COLS);
     }
+}
+
+// Largest number of co-resident pair clusters of this kernel (cached per device and type).
+template <typename OutT>
+static int max_clusters() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) {
+        cudaLaunchConfig_t cfg = {};
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cfg.gridDim = dim3((unsigned)(sms & ~1));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = SMEM_BYTES;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, w2a4_gemm_pair_kernel<OutT>, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sms / 2;
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
 }
 
 template <typename OutT>
@@ -1214,13 +1304,13 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     }
     const cudaError_t e = ensure_smem(w2a4_gemm_pair_kernel<OutT>, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int64_t pairs = (N + 2 * BMW - 1) / (2 * BMW);
-    if (2 * pairs > 0x7fffffff) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)(2 * pairs), (unsigned)((T + BNT - 1) / BNT));
+    const int64_t tiles = ((N + 2 * BMW - 1) / (2 * BMW)) * ((T + BNT - 1) / BNT);
+    if (tiles > 0x3fffffff) return cudaErrorInvalidValue;
+    const int clusters = (int)std::min<int64_t>(tiles, std::max(1, max_clusters<OutT>()));
     const int stall = gemm::g_stall_next ? 1 : 0;
     gemm::g_stall_next = false;
-    w2a4_gemm_pair_kernel<OutT><<<grid, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
-                                                                   gemm::g_wait_limit, stall);
+    w2a4_gemm_pair_kernel<OutT><<<2 * clusters, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N,
+                                                                            (int)K, y, gemm::g_wait_limit, stall);
     return cudaGetLastError();
 }
 
