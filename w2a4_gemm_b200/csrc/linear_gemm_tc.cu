@@ -990,6 +990,12 @@ __device__ __forceinline__ bool wait_fast(uint64_t* bar, uint32_t parity, int* a
     return tc::mbar_try_wait(bar, parity) || gemm::wait_or_abort(bar, parity, abort, limit);
 }
 
+// int32 -> fp32 without the conversion pipe: exact for |v| < 2^22 (|acc| <= 4 * 7 * n_in <= 2^20
+// here), since 1.5 * 2^23 + v is then an fp32 integer and the subtraction is exact.
+__device__ __forceinline__ float i2f_exact(int v) {
+    return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
+}
+
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory"); }
 
 struct Tile {
@@ -1169,10 +1175,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ---------------------------------------------------------------- epilogue
         // Warp (quarter, column group): 32 weight rows, a quarter of each pass's columns.  Per tile:
-        // drain the accumulator (scaled, converted) into the staging buffer in [token][row]
-        // order -- in two passes of 128 columns for fp32 output -- release the accumulator after
-        // the last pass's reads, then write 16-byte pieces along n.  Every epilogue warp runs
-        // every named barrier of every tile, also after an abort (`alive` only skips the work).
+        // drain the accumulator (scaled, converted) into the staging buffer -- fp16 as packed
+        // token pairs [token/2][row][2], fp32 as [token][row] in two passes of 128 columns --
+        // release the accumulator after the last pass's reads, then write 16-byte pieces along n.
+        // The drain stalls the next tile's MMAs, so it keeps off the conversion pipe (exact
+        // integer-to-float by magic number, one packed two-value fp16 conversion).  Every
+        // epilogue warp runs every named barrier of every tile, also after an abort (`alive`
+        // only skips the work).
         constexpr int CPP = STG_BYTES / (BMW * (int)sizeof(OutT));  // columns per pass: 256 / 128
         constexpr int PASSES = BNT / CPP;
         constexpr int EPP = 16 / sizeof(OutT);                      // elements per 16-byte piece
@@ -1201,10 +1210,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         uint32_t acc[32];
                         tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
                         tc::tmem_ld_wait();
+                        if constexpr (sizeof(OutT) == 2) {
+                            uint32_t* stg32 = reinterpret_cast<uint32_t*>(sm.stg);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float v = __fmul_rn(__fmul_rn((float)(int)acc[j], sw), sm.sa[c0 + j]);
-                            gemm_ts::store_one<OutT>(stg + (cl0 + j) * BMW + r, v);
+                            for (int j = 0; j < 32; j += 2) {
+                                const float v0 = __fmul_rn(__fmul_rn(i2f_exact((int)acc[j]), sw), sm.sa[c0 + j]);
+                                const float v1 = __fmul_rn(__fmul_rn(i2f_exact((int)acc[j + 1]), sw), sm.sa[c0 + j + 1]);
+                                const __half2 h = __floats2half2_rn(v0, v1);  // .x = token c0 + j
+                                stg32[((cl0 + j) / 2) * BMW + r] = *reinterpret_cast<const uint32_t*>(&h);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) {
+                                const float v = __fmul_rn(__fmul_rn(i2f_exact((int)acc[j]), sw), sm.sa[c0 + j]);
+                                gemm_ts::store_one<OutT>(stg + (cl0 + j) * BMW + r, v);
+                            }
                         }
                     }
                     if (p == PASSES - 1) {  // every column of the accumulator has been read
@@ -1215,18 +1235,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 epi_bar();  // staging complete
                 if (alive) {
+                    if constexpr (sizeof(OutT) == 2) {
+                        // Piece (token pair jp, 8 rows): 32 staged bytes hold both tokens' halves,
+                        // split with byte permutes into one 16-byte row piece per token.
+                        const uint32_t* stg32 = reinterpret_cast<const uint32_t*>(sm.stg);
 #pragma unroll 2
-                    for (int q = et; q < CPP * PPR; q += kEpiThreads) {
-                        const int j = q / PPR, sub = q % PPR;
-                        const int t = tl.t0 + p * CPP + j, nn = tl.n0 + sub * EPP;
-                        if (t < T) {
-                            OutT* dst = y + (int64_t)t * N + nn;
-                            const OutT* src = stg + j * BMW + sub * EPP;
-                            if (vec_ok && nn + EPP <= N) {
-                                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-                            } else {
-                                for (int e = 0; e < EPP; ++e)
-                                    if (nn + e < N) dst[e] = src[e];
+                        for (int q = et; q < (CPP / 2) * PPR; q += kEpiThreads) {
+                            const int jp = q / PPR, sub = q % PPR;
+                            const int t = tl.t0 + p * CPP + 2 * jp, nn = tl.n0 + sub * EPP;
+                            if (t < T) {
+                                const uint4 u0 = *reinterpret_cast<const uint4*>(stg32 + jp * BMW + sub * 8);
+                                const uint4 u1 = *reinterpret_cast<const uint4*>(stg32 + jp * BMW + sub * 8 + 4);
+                                const uint32_t u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                                uint32_t lo[4], hi[4];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    lo[k] = __byte_perm(u[2 * k], u[2 * k + 1], 0x5410);
+                                    hi[k] = __byte_perm(u[2 * k], u[2 * k + 1], 0x7632);
+                                }
+                                for (int tt = 0; tt < 2 && t + tt < T; ++tt) {
+                                    const uint32_t* w = tt ? hi : lo;
+                                    OutT* dst = y + (int64_t)(t + tt) * N + nn;
+                                    if (vec_ok && nn + EPP <= N) {
+                                        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                                    } else {
+                                        const __half* hv = reinterpret_cast<const __half*>(w);
+                                        for (int e = 0; e < EPP; ++e)
+                                            if (nn + e < N) dst[e] = hv[e];
+                                    }
+                                }
+                            }
+                        }
+                    } else {
+#pragma unroll 2
+                        for (int q = et; q < CPP * PPR; q += kEpiThreads) {
+                            const int j = q / PPR, sub = q % PPR;
+                            const int t = tl.t0 + p * CPP + j, nn = tl.n0 + sub * EPP;
+                            if (t < T) {
+                                OutT* dst = y + (int64_t)t * N + nn;
+                                const OutT* src = stg + j * BMW + sub * EPP;
+                                if (vec_ok && nn + EPP <= N) {
+                                    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                                } else {
+                                    for (int e = 0; e < EPP; ++e)
+                                        if (nn + e < N) dst[e] = src[e];
+                                }
                             }
                         }
                     }
