@@ -2,11 +2,26 @@
 // Arguments are validated by the caller; launchers only configure and launch.
 #pragma once
 
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
 namespace qift {
+
+// The driver's cuTensorMapEncodeTiled (through the runtime's entry-point query, so the library
+// links no libcuda); null if unavailable.
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device), so launches --
 // including ones captured into CUDA graphs -- do not repeat the attribute call.
