@@ -61,8 +61,8 @@ def peaks():
 PROFILED_TRAFFIC = {
     "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="ac7b33485df99f62", bytes=4231168 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
-    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="8c6476ba935a999f",
-                    bytes=19738112 + 2433280, profile="profiles/w2a4_gemm_ts_kernel_mlp_prefill_T2048.md"),
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="5a0db57999d1fc9e",
+                    bytes=19753728 + 1263104, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
     "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="cb37b8ef06a6c6db", bytes=14833152 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
     "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="d77053b1a3d2c13a",
