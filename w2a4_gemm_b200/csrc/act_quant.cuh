@@ -30,11 +30,21 @@ __device__ __forceinline__ float block_max(float v, float* red) {
     return m;
 }
 
+// 4096-point rotation by one CTA: 4096 = 16 x 16 x 16, so three rounds of in-register 16-point
+// butterflies (index bits 0-3, then 4-7, then 8-11) joined by two shared-memory transposes
+// replace the warp-shuffle stages.  The stages still run in the order h = 1, 2, ..., 2048, so
+// every output is the same sequence of fp32 operations.  The buffer is padded by 16 floats per
+// 256 so that both transposes read conflict-free.
+__host__ __device__ constexpr int tpad4096(int a) { return a + ((a >> 8) << 4); }
+constexpr size_t kTbuf4096Bytes = (size_t)(tpad4096(4095) + 1) * sizeof(float);
+
 // Shared memory the rotation needs besides the token itself (transpose buffer).
 template <int LOGB>
 __host__ __device__ constexpr size_t act_tbuf_bytes() {
     if constexpr (LOGB == 0) {
         return 0;
+    } else if constexpr (LOGB == 12) {
+        return kTbuf4096Bytes;
     } else {
         using S = FwhtShape<LOGB>;
         return S::W > 1 ? (size_t)(kActThreads / S::TPS) * S::B * sizeof(float) : 0;
@@ -58,6 +68,34 @@ __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt,
                 const float2 f = __half22float2(h[j]);
                 amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
             }
+        }
+    } else if constexpr (LOGB == 12) {
+        static_assert(kActThreads == 256, "one 16-value column per thread");
+        const int lo = tid & 15, hi = tid >> 4;
+        for (int64_t seg = 0; seg < K / 4096; ++seg) {
+            float v[16];
+            load_contig<16>(xt + seg * 4096 + tid * 16, v);
+            reg_stages<16>(v);  // h = 1 .. 8
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4*>(tbuf + tpad4096(16 * tid + i)) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = tbuf[tpad4096(lo + 16 * i + 256 * hi)];
+            reg_stages<16>(v);  // h = 16 .. 128
+#pragma unroll
+            for (int i = 0; i < 16; ++i) tbuf[tpad4096(lo + 16 * i + 256 * hi)] = v[i];  // same slots as read
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = tbuf[tpad4096(tid + 256 * i)];
+            reg_stages<16>(v);  // h = 256 .. 2048
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const __half h = __float2half_rn(__fmul_rn(v[i], c));
+                amax = fmaxf(amax, fabsf(__half2float(h)));
+                xs[seg * 4096 + tid + 256 * i] = h;
+            }
+            __syncthreads();  // tbuf is reused by the next segment
         }
     } else {
         using S = FwhtShape<LOGB>;
