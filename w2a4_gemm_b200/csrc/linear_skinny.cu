@@ -35,6 +35,7 @@ constexpr int WARPS = 8;
 constexpr int RB = WARPS * 16;  // output rows per cluster
 constexpr int CHUNK_WORDS = 16;  // 256 K values per chunk
 constexpr int PF = 4;            // chunks of codes in flight per lane
+constexpr int RBP = RB + 4;      // padded row stride of the partial sums (conflict-free writes)
 
 __device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -66,7 +67,9 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     extern __shared__ __align__(16) uint8_t smem[];
     const int S = KS + 64;                            // token row stride (== 64 mod 128)
     uint8_t* acts = smem;                             // TP x S bytes
-    int* part = reinterpret_cast<int*>(smem + TP * S);  // RB x TP int32 partial sums
+    int* part = reinterpret_cast<int*>(smem + TP * S);  // [TP][RBP] int32 partial sums
+    float* sa_s = reinterpret_cast<float*>(part + TP * RBP);  // [TP] activation scales
+    float* sw_s = sa_s + TP;                                    // [RB] weight scales of the block
 
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -98,16 +101,34 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     griddep_launch_dependents();
     griddep_wait();
 
-    // Stage this CTA's K slice of every token, permuted to the decode order.
+    // Stage this CTA's K slice of every token, permuted to the decode order (eight loads in
+    // flight per thread before any is used), and the scales the epilogue needs.
     const int groups = KS / 16;
-    for (int i = threadIdx.x; i < TP * groups; i += WARPS * 32) {
-        const int t = i / groups, G = i - t * groups;
-        const int64_t k = (int64_t)kw0 * 16 + (int64_t)G * 16;
-        uint4 a = make_uint4(0u, 0u, 0u, 0u);
-        if (t < T && k + 16 <= K) a = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
-        uint32_t p[4];
-        permute_acts(a, p);
-        *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+    for (int i0 = 0; i0 < TP * groups; i0 += 8 * WARPS * 32) {
+        uint4 a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * WARPS * 32 + threadIdx.x;
+            const int t = i / groups, G = i - t * groups;
+            const int64_t k = (int64_t)kw0 * 16 + (int64_t)G * 16;
+            a[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < TP * groups && t < T && k + 16 <= K) a[u] = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * WARPS * 32 + threadIdx.x;
+            if (i < TP * groups) {
+                const int t = i / groups, G = i - t * groups;
+                uint32_t p[4];
+                permute_acts(a[u], p);
+                *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+            }
+        }
+    }
+    if (threadIdx.x < TP) sa_s[threadIdx.x] = (int)threadIdx.x < T ? s_a[threadIdx.x] : 0.0f;
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + RB) {
+        const int64_t n = (int64_t)row_block * RB + threadIdx.x - 32;
+        sw_s[threadIdx.x - 32] = n < N ? s_w[n] : 0.0f;
     }
     __syncthreads();
 
@@ -144,29 +165,28 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
         }
     }
 
-    // Partial sums of this CTA's K slice: part[row][token].
+    // Partial sums of this CTA's K slice: part[token][row] (row stride RBP: conflict-free).
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int rl = warp * 16 + g, t0 = nt * 8 + 2 * qd;
-        part[rl * TP + t0] = acc[nt][0];
-        part[rl * TP + t0 + 1] = acc[nt][1];
-        part[(rl + 8) * TP + t0] = acc[nt][2];
-        part[(rl + 8) * TP + t0 + 1] = acc[nt][3];
+        part[t0 * RBP + rl] = acc[nt][0];
+        part[(t0 + 1) * RBP + rl] = acc[nt][1];
+        part[t0 * RBP + rl + 8] = acc[nt][2];
+        part[(t0 + 1) * RBP + rl + 8] = acc[nt][3];
     }
     cluster.sync();
 
-    // CTA `rank` finishes rows [rank*RB/C, (rank+1)*RB/C) of the block: add the C partials.
+    // CTA `rank` finishes rows [rank*RB/C, (rank+1)*RB/C) of the block: add the C partials;
+    // consecutive threads take consecutive rows of one token, so the stores run along n.
     const int rows_per = RB / C;
+#pragma unroll 4
     for (int i = threadIdx.x; i < rows_per * TP; i += WARPS * 32) {
-        const int rl = rank * rows_per + i / TP, t = i % TP;
+        const int t = i / rows_per, rl = rank * rows_per + (i - t * rows_per);
         int sum = 0;
-        for (int p = 0; p < C; ++p) {
-            const int* rp = cluster.map_shared_rank(part, p);
-            sum += rp[rl * TP + t];
-        }
+        for (int p = 0; p < C; ++p) sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
         const int64_t n = (int64_t)row_block * RB + rl;
         if (t < T && n < N) {
-            const float v = __fmul_rn(__fmul_rn((float)sum, s_w[n]), s_a[t]);
+            const float v = __fmul_rn(__fmul_rn((float)sum, sw_s[rl]), sa_s[t]);
             store_y<OutT>(y + (int64_t)t * N + n, v);
         }
     }
@@ -182,7 +202,7 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     int C = 1;
     while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
     const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
-    const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)RB * NT * 8 * sizeof(int);
+    const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)NT * 8 * RBP * sizeof(int) + (size_t)(NT * 8 + RB) * 4;
     cudaError_t e = ensure_smem(skinny_kernel<NT, OutT>, smem);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (N + RB - 1) / RB;
