@@ -6,7 +6,9 @@
 // 4-bit activations.  acc[t][n] = sum_k q[t][k] L(code[n][k]) in int32, then the fp32 scales.
 //
 // Work split.  A thread-block cluster of C CTAs shares one block of 128 output rows; CTA r of
-// the cluster owns the K slice [r*KS, (r+1)*KS).  Each of its 8 warps owns 16 rows.  The CTA
+// the cluster owns the K slice [r*KS, (r+1)*KS).  Each 16-row group of the block is owned by
+// one warp, or by two warps taking alternate 256-input chunks when the grid leaves an SM per
+// CTA (more warps in flight per SM; their int32 partials are added in shared memory).  The CTA
 // stages its slice of every token's int8 activations once in shared memory, permuted per
 // 16-byte group to the decode order, so the weights never touch shared memory: a lane loads
 // 16 bytes (4 words = 64 codes) of each of its two rows, decodes a word into four int8x4
@@ -31,8 +33,8 @@ namespace skinny {
 
 namespace cg = cooperative_groups;
 
-constexpr int WARPS = 8;
-constexpr int RB = WARPS * 16;  // output rows per cluster
+constexpr int ROW_WARPS = 8;                    // warps along the rows: 16 rows each
+constexpr int RB = ROW_WARPS * 16;              // output rows per cluster
 constexpr int CHUNK_WORDS = 16;  // 256 K values per chunk
 constexpr int PF = 4;            // chunks of codes in flight per lane
 constexpr int RBP = RB + 4;      // padded row stride of the partial sums (conflict-free writes)
@@ -56,14 +58,17 @@ __device__ __forceinline__ void store_y<float>(float* p, float v) { *p = v; }
 template <>
 __device__ __forceinline__ void store_y<__half>(__half* p, float v) { *p = __float2half_rn(v); }
 
-// NT token tiles of 8 (T <= 8*NT).  KS: K slice per CTA in bytes (multiple of 256).
-template <int NT, typename OutT>
-__global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __restrict__ q,
+// NT token tiles of 8 (T <= 8*NT).  KS: K slice per CTA in bytes (multiple of 256).  KSPLIT
+// warps share each 16-row group, taking alternate K chunks: 2 when the grid has at most one CTA
+// per SM (16 warps hide more latency), 1 otherwise (two CTAs of 8 warps fit on an SM).
+template <int NT, int KSPLIT, typename OutT>
+__global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const int8_t* __restrict__ q,
                                                             const float* __restrict__ s_a,
                                                             const uint32_t* __restrict__ codes,
                                                             const float* __restrict__ s_w, uint32_t lut, int T,
                                                             int N, int K, int KS, OutT* __restrict__ y) {
     constexpr int TP = NT * 8;  // padded tokens
+    constexpr int THREADS = 32 * ROW_WARPS * KSPLIT;
     extern __shared__ __align__(16) uint8_t smem[];
     const int S = KS + 64;                            // token row stride (== 64 mod 128)
     uint8_t* acts = smem;                             // TP x S bytes
@@ -80,7 +85,9 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     const int KW = K / 16;
     const int kw0 = rank * (KS / 16);                  // first word of this CTA's slice
     const int nchunks = KS / 256;
-    const int64_t r_lo = (int64_t)row_block * RB + warp * 16 + g;
+    const int rw = warp % ROW_WARPS, ks = warp / ROW_WARPS;  // row warp, K parity
+    const int my_n = (nchunks - ks + KSPLIT - 1) / KSPLIT;   // this warp's chunks: ks, ks+2, ...
+    const int64_t r_lo = (int64_t)row_block * RB + rw * 16 + g;
     const int64_t r_hi = r_lo + 8;
 
     auto load_chunk = [&](int c, uint4& lo, uint4& hi) {
@@ -97,18 +104,18 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     // ring of PF chunks per lane keeps PF KB of codes per warp in flight.
     uint4 buf[PF][2];
 #pragma unroll
-    for (int u = 0; u < PF; ++u) load_chunk(u, buf[u][0], buf[u][1]);
+    for (int u = 0; u < PF; ++u) load_chunk(ks + KSPLIT * u, buf[u][0], buf[u][1]);
     griddep_launch_dependents();
     griddep_wait();
 
     // Stage this CTA's K slice of every token, permuted to the decode order (eight loads in
     // flight per thread before any is used), and the scales the epilogue needs.
     const int groups = KS / 16;
-    for (int i0 = 0; i0 < TP * groups; i0 += 8 * WARPS * 32) {
+    for (int i0 = 0; i0 < TP * groups; i0 += 8 * THREADS) {
         uint4 a[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * WARPS * 32 + threadIdx.x;
+            const int i = i0 + u * THREADS + threadIdx.x;
             const int t = i / groups, G = i - t * groups;
             const int64_t k = (int64_t)kw0 * 16 + (int64_t)G * 16;
             a[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -116,7 +123,7 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * WARPS * 32 + threadIdx.x;
+            const int i = i0 + u * THREADS + threadIdx.x;
             if (i < TP * groups) {
                 const int t = i / groups, G = i - t * groups;
                 uint32_t p[4];
@@ -138,14 +145,14 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
 
-    for (int c0 = 0; c0 < nchunks; c0 += PF) {
+    for (int i0 = 0; i0 < my_n; i0 += PF) {
 #pragma unroll
         for (int u = 0; u < PF; ++u) {
-            const int c = c0 + u;
-            if (c < nchunks) {
+            const int i = i0 + u, c = ks + KSPLIT * i;
+            if (i < my_n) {
                 const uint32_t wl[4] = {buf[u][0].x, buf[u][0].y, buf[u][0].z, buf[u][0].w};
                 const uint32_t wh[4] = {buf[u][1].x, buf[u][1].y, buf[u][1].z, buf[u][1].w};
-                if (c + PF < nchunks) load_chunk(c + PF, buf[u][0], buf[u][1]);
+                if (i + PF < my_n) load_chunk(c + KSPLIT * PF, buf[u][0], buf[u][1]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint32_t dl[4], dh[4];
@@ -165,14 +172,29 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
         }
     }
 
-    // Partial sums of this CTA's K slice: part[token][row] (row stride RBP: conflict-free).
+    // Partial sums of this CTA's K slice: part[token][row] (row stride RBP: conflict-free).  With
+    // KSPLIT == 2 the odd-chunk warps write and the even-chunk warps of the same rows add theirs.
+    const int rl = rw * 16 + g;
+    if (ks == KSPLIT - 1) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int rl = warp * 16 + g, t0 = nt * 8 + 2 * qd;
-        part[t0 * RBP + rl] = acc[nt][0];
-        part[(t0 + 1) * RBP + rl] = acc[nt][1];
-        part[t0 * RBP + rl + 8] = acc[nt][2];
-        part[(t0 + 1) * RBP + rl + 8] = acc[nt][3];
+        for (int nt = 0; nt < NT; ++nt) {
+            const int t0 = nt * 8 + 2 * qd;
+            part[t0 * RBP + rl] = acc[nt][0];
+            part[(t0 + 1) * RBP + rl] = acc[nt][1];
+            part[t0 * RBP + rl + 8] = acc[nt][2];
+            part[(t0 + 1) * RBP + rl + 8] = acc[nt][3];
+        }
+    }
+    if constexpr (KSPLIT == 2) __syncthreads();
+    if (KSPLIT == 2 && ks == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int t0 = nt * 8 + 2 * qd;
+            part[t0 * RBP + rl] += acc[nt][0];
+            part[(t0 + 1) * RBP + rl] += acc[nt][1];
+            part[t0 * RBP + rl + 8] += acc[nt][2];
+            part[(t0 + 1) * RBP + rl + 8] += acc[nt][3];
+        }
     }
     cluster.sync();
 
@@ -180,7 +202,7 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     // consecutive threads take consecutive rows of one token, so the stores run along n.
     const int rows_per = RB / C;
 #pragma unroll 4
-    for (int i = threadIdx.x; i < rows_per * TP; i += WARPS * 32) {
+    for (int i = threadIdx.x; i < rows_per * TP; i += THREADS) {
         const int t = i / rows_per, rl = rank * rows_per + (i - t * rows_per);
         int sum = 0;
         for (int p = 0; p < C; ++p) sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
@@ -193,22 +215,27 @@ __global__ void __launch_bounds__(WARPS * 32) skinny_kernel(const int8_t* __rest
     cluster.sync();  // keep this CTA's partials alive until every peer has read them
 }
 
-template <int NT, typename OutT>
-static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
-                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
-    // Cluster size: split K so that each CTA streams a slice of at most 2048 inputs (64 KB of
-    // codes for its 128 rows) -- long-lived CTAs, yet enough of them when N is small.  C is a
-    // power of two <= 8, so it divides RB and every CTA finishes a whole number of rows.
-    int C = 1;
-    while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
-    const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
+static int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int v = 0;
+        cached[dev] = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0 ? v : 148;
+    }
+    return cached[dev];
+}
+
+template <int NT, int KSPLIT, typename OutT>
+static cudaError_t launch_k(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, int C, int KS, OutT* y, cudaStream_t s) {
     const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)NT * 8 * RBP * sizeof(int) + (size_t)(NT * 8 + RB) * 4;
-    cudaError_t e = ensure_smem(skinny_kernel<NT, OutT>, smem);
+    cudaError_t e = ensure_smem(skinny_kernel<NT, KSPLIT, OutT>, smem);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (N + RB - 1) / RB;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(blocks * C));
-    cfg.blockDim = dim3(WARPS * 32);
+    cfg.blockDim = dim3(32 * ROW_WARPS * KSPLIT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -220,7 +247,22 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N, (int)K, KS, y);
+    return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, KSPLIT, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N, (int)K,
+                              KS, y);
+}
+
+template <int NT, typename OutT>
+static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
+                            int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    // Cluster size: split K so that each CTA streams a slice of at most 2048 inputs (64 KB of
+    // codes for its 128 rows) -- long-lived CTAs, yet enough of them when N is small.  C is a
+    // power of two <= 8, so it divides RB and every CTA finishes a whole number of rows.
+    int C = 1;
+    while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
+    const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
+    const int64_t ctas = ((N + RB - 1) / RB) * C;
+    if (ctas <= sm_count()) return launch_k<NT, 2, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
+    return launch_k<NT, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
 }
 
 }  // namespace skinny
