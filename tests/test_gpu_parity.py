@@ -134,6 +134,21 @@ def test_quantize_acts_zero_and_tiny_tokens():
         assert np.array_equal(host(gs).view(np.uint32), s.view(np.uint32))
 
 
+# Batches of many tokens take the streaming quantizer (persistent CTAs, registers only): blocks
+# 16..512, widths of one to four 4096-element passes with ragged last passes, zero tokens.
+@pytest.mark.parametrize("block,K", [(16, 1024), (32, 4160), (128, 4096), (128, 11008), (256, 12288),
+                                      (512, 16384), (64, 8256)])
+def test_quantize_acts_many_tokens(block, K):
+    T = 700
+    x = synth.activations(T, K, (T, K, block), n_outliers=synth.outlier_count(K))
+    x[3] = 0
+    x[T - 1] = 0
+    q, s, _ = oracle.quantize_acts(x, block)
+    gq, gs = qg.qift_quantize_acts(dev(x), block)
+    assert np.array_equal(host(gq), q)
+    assert np.array_equal(host(gs).view(np.uint32), s.view(np.uint32))
+
+
 # ---------------------------------------------------------------------------------- linear
 def _linear_case(name, T, N, K, seed, out_dtype):
     rng = np.random.default_rng(seed)
