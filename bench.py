@@ -63,7 +63,7 @@ PROFILED_TRAFFIC = {
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
     "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="5a0db57999d1fc9e",
                     bytes=19753728 + 1263104, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
-    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="cb37b8ef06a6c6db", bytes=14833152 + 0,
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="11e0d18d1b6121e0", bytes=14854144 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
     "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="d77053b1a3d2c13a",
                     bytes=67137024 + 690688, scale=14336 * 4096 / (4096 * 4096),
