@@ -109,6 +109,23 @@ def test_quantize_weights_edge_rows():
             assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
 
 
+def test_quantize_weights_tiny_rows():
+    # Rows small enough that squared errors are subnormal or zero (exact widening fallback),
+    # beside ordinary rows in the same launch.
+    K = 256
+    w = synth.weights(8, K, (77,)) * np.float32(1e-22)
+    w[0] = synth.weights(1, K, (78,))[0]
+    w[1] = 0
+    w[2, ::3] = np.float32(1e-30)
+    w = w.astype(np.float32)
+    for name in ("qift", "pot", "std"):
+        codes, scales, mse, _ = oracle.quantize_weights(w, name)
+        gc, gs, gm = qg.qift_quantize_weights(dev(w), name)
+        assert np.array_equal(codes_u32(gc), codes), name
+        assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+        assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
 # -------------------------------------------------------------------- activation quantizer
 @pytest.mark.parametrize("block", [0, 16, 128, 512, 4096])
 @pytest.mark.parametrize("T,K", [(1, 4096), (3, 512), (16, 11008), (33, 4096)])
