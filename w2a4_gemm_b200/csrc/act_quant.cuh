@@ -151,7 +151,10 @@ __device__ __forceinline__ uint4 quant16(const __half* xs16, float inv) {
         uint32_t word = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            int v = __float2int_rn(__fmul_rn(f[e], inv));
+            // rint (half to even) by the magic-number add, on the fp32 pipe instead of the
+            // conversion unit: exact for |t| < 2^22, and |x * 7/m| <= 7 (1 + 2^-23) here.
+            const float t = __fadd_rn(__fmul_rn(f[e], inv), 12582912.0f);
+            int v = __float_as_int(t) - 0x4B400000;
             v = v > 7 ? 7 : (v < -7 ? -7 : v);
             word |= (uint32_t)(v & 0xff) << (8 * e);
         }
