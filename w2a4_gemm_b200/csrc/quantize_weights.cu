@@ -6,22 +6,23 @@
 // Inference", Abstract: a fixed two-bit code-to-level mapping with the standard per-channel
 // scale (no zero point, no group grid).
 //
-// One CTA owns one output row.  The row is staged in shared memory; thread g evaluates
-// candidate scale s_g by walking the row in index order and accumulating the fp32 squared
+// One CTA owns a few output rows, staged in shared memory; the thread of (row, candidate g)
+// evaluates scale s_g by walking the row in index order and accumulating the fp32 squared
 // error into fp64 -- the fixed order makes the argmin reproducible bit for bit.  This pass is
-// ALU-bound (G candidates x K elements per row), not HBM-bound.
+// ALU-bound (G candidates x K elements per row), not HBM-bound; the fp32 -> fp64 widening, one
+// per evaluation, runs on the conversion unit, which sets the pace.
 //
 // Level thresholds are compared in fp32 against products rounded DOWN: for a float x and a
 // real threshold tau = c*s, x > tau exactly when x > RD(c*s), because no float lies strictly
 // between RD(c*s) and RU(c*s).  That decides every weight exactly as an exact comparison would.
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace qift {
-
-constexpr int kQwThreads = 128;
 
 template <int SET>
 struct Encoder {
@@ -67,47 +68,66 @@ struct Encoder {
     }
 };
 
-template <int SET>
-__global__ void __launch_bounds__(kQwThreads) quant_weights_kernel(const float* __restrict__ w, int64_t K, int G,
-                                                                   double lo, double hi,
-                                                                   uint32_t* __restrict__ codes,
-                                                                   float* __restrict__ scales,
-                                                                   double* __restrict__ row_mse) {
-    extern __shared__ __align__(16) float ws[];  // the row, K floats
-    __shared__ float cand[256];
-    __shared__ double mse[256];
-    __shared__ float red[kQwThreads / 32];
-    __shared__ int best_s;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row = blockIdx.x;
-    const float* wr = w + row * K;
+constexpr int kQwMaxRows = 4;   // rows per CTA
+constexpr int kQwMaxG = 256;     // candidates per row (API limit)
 
-    // Stage the row and find max |w|.
-    float m = 0.0f;
-    for (int64_t i = (int64_t)tid * 4; i < K; i += kQwThreads * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(wr + i);
-        *reinterpret_cast<float4*>(ws + i) = v;
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
+// One CTA owns R <= 4 output rows, staged together in shared memory, so that R x G (row,
+// candidate) pairs -- one per thread -- fill whole warps (G = 100 alone leaves a 128-thread CTA's
+// last warp with 4 busy lanes, and the bottleneck, the conversion unit, is paid per warp).
+template <int SET>
+__global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __restrict__ w, int64_t n_out, int64_t K,
+                                                             int R, int G, double lo, double hi,
+                                                             uint32_t* __restrict__ codes, float* __restrict__ scales,
+                                                             double* __restrict__ row_mse) {
+    extern __shared__ __align__(16) float ws[];  // R rows of K floats
+    __shared__ float cand[kQwMaxRows * kQwMaxG];
+    __shared__ double mse[kQwMaxRows * kQwMaxG];
+    __shared__ float red[kQwMaxRows][32];
+    __shared__ int best_s[kQwMaxRows];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x, nwarps = nthr >> 5;
+    const int64_t row0 = (int64_t)blockIdx.x * R;
+    const int rows = (int)min((int64_t)R, n_out - row0);
+
+    // Stage the rows and find each row's max |w|.
+    float m[kQwMaxRows];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) red[warp] = m;
+    for (int r = 0; r < kQwMaxRows; ++r) {
+        m[r] = 0.0f;
+        if (r < rows) {
+            const float* wr = w + (row0 + r) * K;
+            for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4) {
+                const float4 v = *reinterpret_cast<const float4*>(wr + i);
+                *reinterpret_cast<float4*>(ws + r * K + i) = v;
+                m[r] = fmaxf(m[r], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m[r] = fmaxf(m[r], __shfl_xor_sync(0xffffffffu, m[r], o));
+        if (lane == 0) red[r][warp] = m[r];
+    }
     __syncthreads();
-    m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    if (tid < kQwMaxRows) {
+        float v = 0.0f;
+        for (int i = 0; i < nwarps; ++i) v = fmaxf(v, red[tid][i]);
+        red[tid][0] = v;
+    }
+    __syncthreads();
 
     // Candidate scales, binary64 in the order lo + ((hi - lo) * k) / (G - 1), then * m / L.
     const double lambda = SET == kSetQift ? 1.5 : (SET == kSetPot ? 4.0 : 2.0);
-    for (int g = tid; g < G; g += kQwThreads) {
-        const double f = __dadd_rn(lo, __ddiv_rn(__dmul_rn(__dsub_rn(hi, lo), (double)g), (double)(G - 1)));
-        cand[g] = __double2float_rn(__ddiv_rn(__dmul_rn(f, (double)m), lambda));
+    for (int f = tid; f < rows * G; f += nthr) {
+        const int r = f / G, g = f - r * G;
+        const double fr = __dadd_rn(lo, __ddiv_rn(__dmul_rn(__dsub_rn(hi, lo), (double)g), (double)(G - 1)));
+        cand[r * kQwMaxG + g] = __double2float_rn(__ddiv_rn(__dmul_rn(fr, (double)red[r][0]), lambda));
     }
     __syncthreads();
 
-    // MSE of every candidate: sequential over the row, fp32 squared error widened to fp64.
-    for (int g = tid; g < G; g += kQwThreads) {
-        const Encoder<SET> enc(cand[g]);
+    // MSE of every (row, candidate): sequential over the row, fp32 squared error widened to fp64.
+    for (int f = tid; f < rows * G; f += nthr) {
+        const int r = f / G, g = f - r * G;
+        const Encoder<SET> enc(cand[r * kQwMaxG + g]);
         double acc = 0.0;
-        const float4* w4 = reinterpret_cast<const float4*>(ws);
+        const float4* w4 = reinterpret_cast<const float4*>(ws + r * K);
         for (int64_t i = 0; i < K / 4; ++i) {
             const float4 v = w4[i];
             acc = __dadd_rn(acc, (double)enc.sq_err(v.x));
@@ -115,53 +135,61 @@ __global__ void __launch_bounds__(kQwThreads) quant_weights_kernel(const float* 
             acc = __dadd_rn(acc, (double)enc.sq_err(v.z));
             acc = __dadd_rn(acc, (double)enc.sq_err(v.w));
         }
-        mse[g] = acc;
+        mse[r * kQwMaxG + g] = acc;
     }
     __syncthreads();
 
-    // Argmin, first index on ties.
-    if (tid == 0) {
+    // Argmin per row, first index on ties.
+    if (tid < rows) {
+        const double* mr = mse + tid * kQwMaxG;
         int b = 0;
-        double bv = mse[0];
+        double bv = mr[0];
         for (int g = 1; g < G; ++g)
-            if (mse[g] < bv) { bv = mse[g]; b = g; }
-        best_s = b;
+            if (mr[g] < bv) { bv = mr[g]; b = g; }
+        best_s[tid] = b;
     }
     __syncthreads();
-    const int b = best_s;
-    const float s = cand[b];
-    const Encoder<SET> enc(s);
 
     // Encode and pack: word j holds the codes of inputs 16j .. 16j+15, 2 bits each.
-    uint32_t* crow = codes + row * (K / 16);
-    for (int64_t j = tid; j < K / 16; j += kQwThreads) {
-        const float4* w4 = reinterpret_cast<const float4*>(ws + j * 16);
-        uint32_t word = 0;
+    for (int r = 0; r < rows; ++r) {
+        const int b = best_s[r];
+        const float sr = cand[r * kQwMaxG + b];
+        const Encoder<SET> enc(sr);
+        uint32_t* crow = codes + (row0 + r) * (K / 16);
+        for (int64_t j = tid; j < K / 16; j += nthr) {
+            const float4* w4 = reinterpret_cast<const float4*>(ws + r * K + j * 16);
+            uint32_t word = 0;
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
-            const float4 v = w4[v4];
-            word |= enc.code(v.x) << (8 * v4);
-            word |= enc.code(v.y) << (8 * v4 + 2);
-            word |= enc.code(v.z) << (8 * v4 + 4);
-            word |= enc.code(v.w) << (8 * v4 + 6);
+            for (int v4 = 0; v4 < 4; ++v4) {
+                const float4 v = w4[v4];
+                word |= enc.code(v.x) << (8 * v4);
+                word |= enc.code(v.y) << (8 * v4 + 2);
+                word |= enc.code(v.z) << (8 * v4 + 4);
+                word |= enc.code(v.w) << (8 * v4 + 6);
+            }
+            crow[j] = word;
         }
-        crow[j] = word;
-    }
-    if (tid == 0) {
-        scales[row] = SET == kSetQift ? __fmul_rn(s, 0.5f) : s;
-        if (row_mse) row_mse[row] = __ddiv_rn(mse[b], (double)K);
+        if (tid == 0) {
+            scales[row0 + r] = SET == kSetQift ? __fmul_rn(sr, 0.5f) : sr;
+            if (row_mse) row_mse[row0 + r] = __ddiv_rn(mse[r * kQwMaxG + b], (double)K);
+        }
     }
 }
 
 template <int SET>
 static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
                              uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
-    const size_t smem = (size_t)n_in * sizeof(float);
+    // As many rows per CTA as fit in ~100 KB of shared memory (so several CTAs share an SM).
+    int R = (int)std::min<int64_t>(kQwMaxRows, std::max<int64_t>(1, (100 * 1024) / (n_in * 4)));
+    const int threads = std::max(128, std::min(1024, (R * G + 31) / 32 * 32));
+    const size_t smem = (size_t)R * n_in * sizeof(float);
     {
         const cudaError_t e = ensure_smem(quant_weights_kernel<SET>, smem);
         if (e != cudaSuccess) return e;
     }
-    quant_weights_kernel<SET><<<(unsigned)n_out, kQwThreads, smem, s>>>(w, n_in, G, lo, hi, codes, scales, row_mse);
+    const int64_t grid = (n_out + R - 1) / R;
+    quant_weights_kernel<SET><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes, scales,
+                                                                    row_mse);
     return cudaGetLastError();
 }
 
