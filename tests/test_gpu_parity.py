@@ -223,6 +223,47 @@ def test_single_linear_256x512_end_to_end():
     assert np.array_equal(host(gy), ref["y"])
 
 
+# ------------------------------------------------- one token (codes bulk-copied on chip)
+@pytest.mark.parametrize("pin", ["auto", "one_token"])
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("N,K", [(1, 64), (37, 64), (147, 128), (149, 640), (300, 4096), (4096, 4096), (1000, 11008),
+                                 (257, 14336), (14336, 4096), (4096, 14336), (5, 16384), (28000, 4096)])
+def test_linear_one_token_parity(pin, name, N, K):
+    # N < SMs (one row per CTA), ragged rows per CTA, slices of 32 groups that do not divide a
+    # row (K = 11008, 14336, 640), and a matrix tall enough to take two CTAs per SM (28000).
+    qg.qift_debug_set_linear_path(pin)
+    try:
+        for out_dtype in (torch.float16, torch.float32):
+            got, ref = _linear_case(name, 1, N, K, 3 * N + K, out_dtype)
+            assert np.array_equal(got.view(np.uint16 if out_dtype == torch.float16 else np.uint32),
+                                  ref.view(np.uint16 if out_dtype == torch.float16 else np.uint32)), (N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
+def test_linear_one_token_extreme_accumulators():
+    # |acc| = 7 * 4 * 16384 (PoT) with every code value, and activations of both signs: the
+    # Qift path applies the codes through masks (bytes up to 0xC0, unsigned) and 2 sum qc - 3 sum q.
+    N, K = 8, 16384
+    codes = np.zeros((N, K // 16), np.uint32)
+    codes[0], codes[1], codes[2], codes[3] = 0xFFFFFFFF, 0, 0xAAAAAAAA, 0x55555555
+    codes[4], codes[5] = 0x1B1B1B1B, 0xE4E4E4E4   # codes 3,2,1,0 / 0,1,2,3 in every byte
+    codes[6] = np.random.default_rng(1).integers(0, 2 ** 32, K // 16, dtype=np.uint64).astype(np.uint32)
+    s_w = np.full(N, 1.0, np.float32)
+    s_a = np.full(1, 1.0, np.float32)
+    for qv in (7, -7, None):
+        q = np.full((1, K), 7 if qv is None else qv, np.int8)
+        if qv is None:
+            q[0, 1::2] = -7
+        for name, top in (("qift", 3), ("pot", 4)):
+            y, acc = oracle.linear(q, s_a, codes, s_w, name, np.float32)
+            if qv is not None:
+                assert np.abs(acc).max() == 7 * top * K
+            gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), name, torch.float32)
+            assert np.array_equal(host(gy), y), (qv, name)
+
+
 # ------------------------------------------------------------- tensor-core GEMM (prefill)
 @pytest.mark.parametrize("path", ["gemm", "gemm_ts", "gemm_tsp", "gemm_pair"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
@@ -272,7 +313,9 @@ def test_pinned_family_rejects_unsupported_shape():
 # ---------------------------------------------------------- one-launch decode (fused a3-a5)
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K,block", [(1, 4096, 4096, 4096), (1, 37, 64, 16), (2, 300, 512, 128), (3, 129, 11008, 128),
-                                          (4, 64, 14336, 128), (1, 1, 1024, 0), (4, 200, 2048, 2048), (1, 5000, 512, 512)])
+                                          (4, 64, 14336, 128), (1, 1, 1024, 0), (4, 200, 2048, 2048), (1, 5000, 512, 512),
+                                          (1, 14336, 4096, 4096), (1, 300, 11008, 128), (1, 4096, 14336, 128),
+                                          (1, 149, 8192, 2048), (1, 28000, 4096, 128)])
 def test_decode_linear_matches_oracle(name, T, N, K, block):
     rng = np.random.default_rng(T * 7 + N + K)
     x = synth.activations(T, K, (T, N, K), n_outliers=synth.outlier_count(K))
@@ -289,6 +332,24 @@ def test_decode_linear_matches_oracle(name, T, N, K, block):
                               ref.view(np.uint16 if npdt == np.float16 else np.uint32))
         assert np.array_equal(host(gq), q)
         assert np.array_equal(host(gsa).view(np.uint32), s_a.view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("N,K,block", [(4096, 4096, 4096), (300, 512, 128)])
+def test_decode_linear_one_token_pinned_to_warp_per_row(name, N, K, block):
+    # Any pin other than auto / one_token sends a one-token decode to the warp-per-row kernel.
+    rng = np.random.default_rng(N + K)
+    x = synth.activations(1, K, (N, K), n_outliers=synth.outlier_count(K))
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 16), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    q, s_a, _ = oracle.quantize_acts(x, block)
+    ref, _ = oracle.linear(q, s_a, codes, s_w, name, np.float16)
+    qg.qift_debug_set_linear_path("gemv")
+    try:
+        gy = qg.qift_decode_linear(dev(x), block, dev(codes.view(np.int32)), dev(s_w), name, torch.float16)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert np.array_equal(host(gy).view(np.uint16), ref.view(np.uint16))
 
 
 def test_decode_linear_zero_token_and_unsupported():

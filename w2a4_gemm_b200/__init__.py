@@ -50,12 +50,14 @@ def lib() -> C.CDLL:
         L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
         L.qift_debug_set_wait_limit.argtypes = [i64]
         L.qift_debug_stall_next_gemm.argtypes = []
+        L.qift_debug_stall_next_one_token.argtypes = []
         L.qift_debug_set_linear_path.argtypes = [i32]
         L.qift_debug_set_pdl.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
+                     "qift_debug_stall_next_one_token",
                      "qift_debug_set_linear_path", "qift_debug_set_pdl"):
             getattr(L, name).restype = C.c_int
         _lib = L
@@ -188,7 +190,8 @@ def qift_device_error(stream=None) -> tuple[int, int]:
 
 
 def qift_debug_set_wait_limit(cycles: int) -> None:
-    """Test hook: SM-cycle limit of every on-chip wait in later tensor-core GEMMs (<= 0: default)."""
+    """Test hook: SM-cycle limit of every on-chip wait in later tensor-core GEMM and one-token
+    launches (<= 0: default)."""
     _check(lib().qift_debug_set_wait_limit(int(cycles)), "qift_debug_set_wait_limit")
 
 
@@ -197,7 +200,13 @@ def qift_debug_stall_next_gemm() -> None:
     _check(lib().qift_debug_stall_next_gemm(), "qift_debug_stall_next_gemm")
 
 
-LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3, "gemm_ts": 4, "gemm_tsp": 5, "gemm_pair": 6}
+def qift_debug_stall_next_one_token() -> None:
+    """Test hook: the next one-token launch waits on a barrier nothing arrives on and times out."""
+    _check(lib().qift_debug_stall_next_one_token(), "qift_debug_stall_next_one_token")
+
+
+LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3, "gemm_ts": 4, "gemm_tsp": 5, "gemm_pair": 6,
+                "one_token": 7}
 
 
 def qift_debug_set_linear_path(path) -> None:

@@ -10,23 +10,26 @@
 
 namespace qift {
 
-constexpr int kActThreads = 256;  // every function below needs all 256 threads of the CTA
+// Every function below runs on 256 threads: the whole CTA (Bar = CtaSync) or threads 0..255 of
+// a larger one (Bar = GroupSync<256>).
+constexpr int kActThreads = 256;
 
+template <typename Bar = CtaSync>
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) red[warp] = v;
-    __syncthreads();
+    Bar::sync();
     if (warp == 0) {
         v = lane < (kActThreads / 32) ? red[lane] : 0.0f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
         if (lane == 0) red[0] = v;
     }
-    __syncthreads();
+    Bar::sync();
     const float m = red[0];
-    __syncthreads();  // red may be reused right after
+    Bar::sync();  // red may be reused right after
     return m;
 }
 
@@ -53,7 +56,7 @@ __host__ __device__ constexpr size_t act_tbuf_bytes() {
 
 // Rotate one token (K fp16 values at xt, K % 16 == 0) into xs as fp16 and return max |x'|.
 // LOGB == 0: the token is already rotated (copied as is).  `red` holds kActThreads/32 floats.
-template <int LOGB>
+template <int LOGB, typename Bar = CtaSync>
 __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt, int64_t K, float c, __half* xs,
                                                   float* tbuf, float* red) {
     const int tid = threadIdx.x, lane = tid & 31;
@@ -79,13 +82,13 @@ __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt,
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
                 *reinterpret_cast<float4*>(tbuf + tpad4096(16 * tid + i)) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            __syncthreads();
+            Bar::sync();
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = tbuf[tpad4096(lo + 16 * i + 256 * hi)];
             reg_stages<16>(v);  // h = 16 .. 128
 #pragma unroll
             for (int i = 0; i < 16; ++i) tbuf[tpad4096(lo + 16 * i + 256 * hi)] = v[i];  // same slots as read
-            __syncthreads();
+            Bar::sync();
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = tbuf[tpad4096(tid + 256 * i)];
             reg_stages<16>(v);  // h = 256 .. 2048
@@ -95,7 +98,7 @@ __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt,
                 amax = fmaxf(amax, fabsf(__half2float(h)));
                 xs[seg * 4096 + tid + 256 * i] = h;
             }
-            __syncthreads();  // tbuf is reused by the next segment
+            Bar::sync();  // tbuf is reused by the next segment
         }
     } else {
         using S = FwhtShape<LOGB>;
@@ -114,7 +117,7 @@ __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt,
                 for (int i = 0; i < S::E; ++i) v[i] = 0.0f;
             }
             float out[S::W][S::R];
-            fwht_segment<LOGB>(v, ts, lane, c, tbuf + (S::W > 1 ? seg_local * S::B : 0), out);
+            fwht_segment<LOGB, Bar>(v, ts, lane, c, tbuf + (S::W > 1 ? seg_local * S::B : 0), out);
             if (active) {
 #pragma unroll
                 for (int j = 0; j < S::W; ++j) {
@@ -127,11 +130,11 @@ __device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt,
                     store_contig<S::R>(xs + seg * S::B + ts * S::R + j * S::COL, hv);
                 }
             }
-            if constexpr (S::W > 1) __syncthreads();  // tbuf is reused by the next pass
+            if constexpr (S::W > 1) Bar::sync();  // tbuf is reused by the next pass
         }
     }
-    __syncthreads();
-    return block_max(amax, red);
+    Bar::sync();
+    return block_max<Bar>(amax, red);
 }
 
 // Sixteen fp16 values -> sixteen INT4 codes in int8 bytes, natural order:

@@ -116,14 +116,20 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
             path = qift::kPathGemmPair;
         else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
             path = qift::kPathSkinny;
+        else if (tokens == 1 && qift::linear_one_token_preferred(n_out, n_in))
+            path = qift::kPathOneToken;
         else
             path = qift::kPathGemv;
     } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs || path == qift::kPathGemmTsp ||
                  path == qift::kPathGemmPair) &&
                 !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
-               (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))) {
+               (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in)) ||
+               (path == qift::kPathOneToken && (tokens != 1 || !qift::linear_one_token_supported(n_out, n_in)))) {
         return QIFT_ERR_UNSUPPORTED;
     }
+    if (path == qift::kPathOneToken)
+        return from_cuda(qift::launch_linear_one_token(q_act, act_scale, codes, w_scale, (int)set, n_out, n_in, y, f16,
+                                                       s));
     if (path == qift::kPathGemmPair)
         return from_cuda(qift::launch_linear_gemm_pair(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
                                                        n_in, y, f16, s));
@@ -156,6 +162,12 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
     if (!aligned16(x) || !aligned16(codes) || !aligned16(y) || !aligned4(w_scale)) return QIFT_ERR_INVALID_ARG;
     if ((q_out && !aligned16(q_out)) || (act_scale_out && !aligned4(act_scale_out))) return QIFT_ERR_INVALID_ARG;
     if (n_out > 0x7fffffff / 2) return QIFT_ERR_UNSUPPORTED;
+    const int path = qift::debug_linear_path();
+    if (tokens == 1 && (path == qift::kPathAuto || path == qift::kPathOneToken) &&
+        qift::decode_one_token_supported(n_out, n_in, block))
+        return from_cuda(qift::launch_decode_one_token(x, n_in, block, codes, w_scale, (int)set, n_out, y,
+                                                       out_dt == QIFT_F16, q_out, act_scale_out,
+                                                       static_cast<cudaStream_t>(stream)));
     return from_cuda(qift::launch_decode_linear(x, tokens, n_in, block, codes, w_scale, (int)set, n_out, y,
                                                 out_dt == QIFT_F16, q_out, act_scale_out,
                                                 static_cast<cudaStream_t>(stream)));
@@ -164,19 +176,22 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
 qift_status qift_device_error(void* stream, int32_t* detail) {
     if (detail) *detail = 0;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QIFT_ERR_CUDA;
-    int word = 0;
+    int word = 0, word1 = 0;
     if (qift::read_and_clear_device_error(&word) != cudaSuccess) return QIFT_ERR_CUDA;
+    if (qift::read_and_clear_one_token_error(&word1) != cudaSuccess) return QIFT_ERR_CUDA;
+    word |= word1;
     if (detail) *detail = word;
     return word ? QIFT_ERR_TIMEOUT : QIFT_OK;
 }
 
 qift_status qift_debug_set_wait_limit(int64_t cycles) {
     qift::debug_set_gemm_wait_limit((long long)cycles);
+    qift::debug_set_one_token_wait_limit((long long)cycles);
     return QIFT_OK;
 }
 
 qift_status qift_debug_set_linear_path(int32_t path) {
-    if (path < 0 || path > 6) return QIFT_ERR_INVALID_ARG;
+    if (path < 0 || path > 7) return QIFT_ERR_INVALID_ARG;
     qift::debug_set_linear_path(path);
     return QIFT_OK;
 }
@@ -188,6 +203,11 @@ qift_status qift_debug_set_pdl(int32_t enable) {
 
 qift_status qift_debug_stall_next_gemm(void) {
     qift::debug_stall_next_gemm();
+    return QIFT_OK;
+}
+
+qift_status qift_debug_stall_next_one_token(void) {
+    qift::debug_stall_next_one_token();
     return QIFT_OK;
 }
 

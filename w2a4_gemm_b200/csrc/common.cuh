@@ -86,11 +86,31 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
     return v;
 }
 
+// Ask L2 for the 128-byte lines of [p, p + bytes), one line per thread of the CTA.  Only a
+// hint: L2 is where global writes become coherent, so a line fetched before the producer of p
+// has finished is updated in place by its writes, and loads after griddep_wait() see them.
+__device__ __forceinline__ void prefetch_l2_cta(const void* p, int64_t bytes) {
+    const char* b = static_cast<const char*>(p);
+    for (int64_t off = (int64_t)threadIdx.x * 128; off < bytes; off += (int64_t)blockDim.x * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+}
+
 // Programmatic dependent launch.  wait: block until the kernels this launch depends on have
 // completed and their writes are visible (a no-op without a programmatic dependency).
 // launch_dependents: allow the next kernel on the stream to start launching.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+// Barrier policies for device code that a whole CTA, or only its first N threads, runs.
+struct CtaSync {
+    __device__ __forceinline__ static void sync() { __syncthreads(); }
+};
+// Named barrier 1 over threads 0 .. N-1 (N a multiple of 32); the other threads must not use
+// barrier 1 meanwhile.
+template <int N>
+struct GroupSync {
+    __device__ __forceinline__ static void sync() { asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory"); }
+};
 
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
 

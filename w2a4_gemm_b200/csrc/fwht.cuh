@@ -142,10 +142,10 @@ __device__ __forceinline__ void store_contig(__half* __restrict__ p, const float
 // Transform one segment owned by TPS consecutive threads.  On entry v holds the thread's E
 // contiguous inputs (elements ts*E .. ts*E+E-1).  On exit out[j][r] is the normalised output
 // element ts*R + r + j*COL, i.e. W runs of R contiguous elements (one run of E when W == 1).
-// `tbuf` is this segment's B-float shared buffer (only used when W > 1); every thread of the
-// CTA must call this function the same number of times, and the caller must __syncthreads()
-// before reusing tbuf.
-template <int LOGB>
+// `tbuf` is this segment's B-float shared buffer (only used when W > 1); every thread that
+// Bar synchronises must call this function the same number of times, and the caller must
+// synchronise them again before reusing tbuf.
+template <int LOGB, typename Bar = CtaSync>
 __device__ __forceinline__ void fwht_segment(float (&v)[FwhtShape<LOGB>::E], int ts, int lane, float c,
                                              float* tbuf,
                                              float (&out)[FwhtShape<LOGB>::W][FwhtShape<LOGB>::R]) {
@@ -159,7 +159,7 @@ __device__ __forceinline__ void fwht_segment(float (&v)[FwhtShape<LOGB>::E], int
 #pragma unroll
         for (int i = 0; i < S::E; i += 4)
             *reinterpret_cast<float4*>(tbuf + ts * S::E + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        __syncthreads();
+        Bar::sync();
 #pragma unroll
         for (int r = 0; r < S::R; ++r) {
             float u[S::W];

@@ -65,8 +65,31 @@ cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t
                                int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                cudaStream_t s);
 
+// One token: qift_linear, and the fused decode step, on CTAs that bulk-copy their rows'
+// codes into shared memory before waiting for the previous kernel (half an SM each).
+bool linear_one_token_supported(int64_t n_out, int64_t n_in);
+bool linear_one_token_preferred(int64_t n_out, int64_t n_in);  // over the warp-per-row GEMV
+bool decode_one_token_supported(int64_t n_out, int64_t n_in, int block);
+cudaError_t launch_linear_one_token(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                    int set, int64_t n_out, int64_t n_in, void* y, bool f16, cudaStream_t s);
+cudaError_t launch_decode_one_token(const void* x, int64_t n_in, int block, const uint32_t* codes, const float* s_w,
+                                    int set, int64_t n_out, void* y, bool f16, int8_t* q_out, float* sa_out,
+                                    cudaStream_t s);
+void debug_set_one_token_wait_limit(long long cycles);
+void debug_stall_next_one_token();
+cudaError_t read_and_clear_one_token_error(int* word);
+
 // Test hooks behind qift_debug.h.
-enum LinearPath { kPathAuto = 0, kPathGemv = 1, kPathSkinny = 2, kPathGemm = 3, kPathGemmTs = 4, kPathGemmTsp = 5, kPathGemmPair = 6 };
+enum LinearPath {
+    kPathAuto = 0,
+    kPathGemv = 1,
+    kPathSkinny = 2,
+    kPathGemm = 3,
+    kPathGemmTs = 4,
+    kPathGemmTsp = 5,
+    kPathGemmPair = 6,
+    kPathOneToken = 7
+};
 void debug_set_linear_path(int path);
 int debug_linear_path();
 void debug_set_pdl(bool on);

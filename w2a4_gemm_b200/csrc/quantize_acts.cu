@@ -25,8 +25,10 @@ __global__ void __launch_bounds__(kActThreads) quant_acts_kernel(const __half* _
     float* tbuf = reinterpret_cast<float*>(smem_raw + ((K * 2 + 15) / 16) * 16);
     const int tid = threadIdx.x;
     const int64_t token = blockIdx.x;
-    // Launched as a programmatic dependent: wait for the previous kernel on the stream before
-    // touching memory, then let the next one (the linear) start its weight stream early.
+    // Launched as a programmatic dependent: the token's lines are requested into L2 while the
+    // previous kernel on the stream finishes; the values are read only after waiting for it.
+    // Then the next kernel (the linear) may start its weight stream early.
+    prefetch_l2_cta(x + token * K, K * 2);
     griddep_wait();
     griddep_launch_dependents();
 
