@@ -111,12 +111,14 @@ qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int3
  *               exact).  tokens == 0 or n_out == 0 is a no-op.
  * Decode-size batches (tokens <= 16) run as an HBM-streaming GEMV; larger batches as an int8
  * tensor-core GEMM (n_in % 64 == 0; otherwise the GEMV).  Both give bit-identical results.
- * Overlap: the decode GEMV is launched as a programmatic dependent of the previous kernel on
- * `stream` and may start reading `codes` -- and only `codes` -- before that kernel has
- * finished; q_act, act_scale, w_scale and y are touched only after it has completed.  So the
- * kernel launched immediately before qift_linear on the same stream must not write `codes`
- * (the usual order qift_quantize_weights -> qift_quantize_acts -> qift_linear satisfies
- * this: qift_quantize_acts waits for its predecessor before it lets qift_linear start).
+ * Overlap: the decode kernels are launched as programmatic dependents of the previous kernel
+ * on `stream` and may start reading the weights -- `codes` and `w_scale`, nothing else --
+ * before that kernel has finished; the values of q_act and act_scale are read, and y written,
+ * only after it has completed (their cache lines may be prefetched into L2 before, which
+ * changes no value).  So the kernel launched immediately before qift_linear on the same stream
+ * must not write `codes` or `w_scale` (the usual order qift_quantize_weights ->
+ * qift_quantize_acts -> qift_linear satisfies this: qift_quantize_acts waits for its
+ * predecessor before it lets qift_linear start).
  */
 qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint32_t* codes,
                         const float* w_scale, qift_levelset set, int64_t tokens, int64_t n_out,
@@ -133,8 +135,8 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
  *   codes, w_scale, set (QIFT or POT), n_out, y, out_dt: as in qift_linear.
  *   q_out       : int8 [tokens][n_in] or NULL -- receives the INT4 activations.
  *   act_scale_out: fp32 [tokens] or NULL -- receives s_a.
- * Like the decode GEMV it may read `codes` before the kernel launched just before it on the
- * same stream has finished, so that kernel must not write `codes`.
+ * Like the decode GEMV it may read `codes` and `w_scale` before the kernel launched just before
+ * it on the same stream has finished, so that kernel must not write them.
  */
 qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int32_t block, const uint32_t* codes,
                                const float* w_scale, qift_levelset set, int64_t n_out, void* y, qift_dtype out_dt,

@@ -121,13 +121,14 @@ __device__ __forceinline__ int dot_group(uint4 wv, const uint4 (&a)[4]) {
 }
 
 // Shared memory after the static part: codes [R][K/64] x 16 B, arranged activations
-// [4][K/64] x 16 B, row sums [R rounded to 4], and for ROT the rotated fp16 token + the
-// rotation's transpose buffer.
+// [4][K/64] x 16 B, row sums and row scales [R rounded to 4] each, and for ROT the rotated fp16
+// token + the rotation's transpose buffer.
 __host__ __device__ inline size_t code_bytes(int64_t R, int64_t K) { return (size_t)R * (size_t)(K / 4); }
 __host__ __device__ inline size_t rowacc_offset(int64_t R, int64_t K) { return code_bytes(R, K) + (size_t)K; }
-__host__ __device__ inline size_t xs_offset(int64_t R, int64_t K) {
+__host__ __device__ inline size_t sw_offset(int64_t R, int64_t K) {
     return rowacc_offset(R, K) + (size_t)((R + 3) & ~3) * 4;
 }
+__host__ __device__ inline size_t xs_offset(int64_t R, int64_t K) { return sw_offset(R, K) + (size_t)((R + 3) & ~3) * 4; }
 
 template <bool ROT, int LOGB, int SET, typename OutT>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -150,8 +151,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint4* cs = reinterpret_cast<const uint4*>(smem);
     uint4* as = reinterpret_cast<uint4*>(smem + code_bytes(R, K));
     int* row_acc = reinterpret_cast<int*>(smem + rowacc_offset(R, K));
+    float* sw_s = reinterpret_cast<float*>(smem + sw_offset(R, K));
 
-    // 1. Before the wait: the barrier, this CTA's codes in flight, x's lines into L2.
+    // 1. Before the wait: the barrier, this CTA's codes in flight, its weight scales, the
+    //    activations' lines into L2.
     if (tid == 0) {
         tc::mbar_init(&bar, 1);
         tc::mbar_init(&never_bar, 1);
@@ -159,7 +162,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         qsum = 0;
         never = 0;
     }
-    for (int i = tid; i < nrows; i += kThreads) row_acc[i] = 0;
+    for (int i = tid; i < nrows; i += kThreads) {
+        row_acc[i] = 0;
+        sw_s[i] = __ldg(s_w + r0 + i);
+    }
     __syncthreads();
     const uint32_t bytes = (uint32_t)code_bytes(nrows, K);
     if (tid == 0 && bytes) {
@@ -225,11 +231,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint4 a[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) a[u] = ch < CPR ? as[u * CPR + ch] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll 4
-        for (int row = rg; row < nrows; row += RG) {
-            int v = ch < CPR ? dot_group<SET>(cs[row * CPR + ch], a) : 0;
-            v = __reduce_add_sync(0xffffffffu, v);
-            if (lane == 0) atomicAdd(&row_acc[row], v);
+        for (int row0 = rg; row0 < nrows; row0 += 4 * RG) {  // four independent rows per pass
+            int v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int row = row0 + j * RG;
+                v[j] = row < nrows && ch < CPR ? dot_group<SET>(cs[row * CPR + ch], a) : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int row = row0 + j * RG;  // warp-uniform
+                const int t = __reduce_add_sync(0xffffffffu, v[j]);
+                if (lane == 0 && row < nrows) atomicAdd(&row_acc[row], t);
+            }
         }
     }
     __syncthreads();
@@ -247,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 4. Epilogue: y = ((float)acc * s_w) * s_a.
     for (int t = tid; t < nrows; t += kThreads) {
         const int acc = SET == kSetQift ? 2 * row_acc[t] - 3 * qsum : row_acc[t];
-        store_out<OutT>(y + r0 + t, __fmul_rn(__fmul_rn((float)acc, __ldg(s_w + r0 + t)), sa_s));
+        store_out<OutT>(y + r0 + t, __fmul_rn(__fmul_rn((float)acc, sw_s[t]), sa_s));
     }
 }
 
