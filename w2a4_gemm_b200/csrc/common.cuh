@@ -86,12 +86,23 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
     return v;
 }
 
-// Ask L2 for the 128-byte lines of [p, p + bytes), one line per thread of the CTA.  Only a
-// hint: L2 is where global writes become coherent, so a line fetched before the producer of p
-// has finished is updated in place by its writes, and loads after griddep_wait() see them.
+// Ask L2 for the 128-byte lines of [p, p + bytes), one line per thread of the CTA (data that
+// only this CTA reads).  A hint only -- see prefetch_l2_grid.
 __device__ __forceinline__ void prefetch_l2_cta(const void* p, int64_t bytes) {
     const char* b = static_cast<const char*>(p);
     for (int64_t off = (int64_t)threadIdx.x * 128; off < bytes; off += (int64_t)blockDim.x * 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+}
+
+// Ask L2 for the 128-byte lines of [p, p + bytes) that every CTA reads, each line once across
+// the grid: thread t of
+// CTA b takes lines (b + t * G), (b + t * G) + G * blockDim, ...  Only a hint: L2 is where
+// global writes become coherent, so a line fetched before the producer of p has finished is
+// updated in place by its writes, and loads after griddep_wait() see them.
+__device__ __forceinline__ void prefetch_l2_grid(const void* p, int64_t bytes) {
+    const char* b = static_cast<const char*>(p);
+    const int64_t G = gridDim.x, step = G * blockDim.x * 128;
+    for (int64_t off = ((int64_t)blockIdx.x + (int64_t)threadIdx.x * G) * 128; off < bytes; off += step)
         asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
 }
 

@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
     };
     // 1. weights first (and x's lines into L2), then wait for the producer of x.
     load_decode(0);
-    prefetch_l2_cta(x, (int64_t)T * K * 2);
+    prefetch_l2_grid(x, (int64_t)T * K * 2);
     griddep_launch_dependents();
     griddep_wait();
     float sw[RMAX];

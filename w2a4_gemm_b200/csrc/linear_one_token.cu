@@ -175,10 +175,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             bulk_g2s(smem + off, src + off, bytes - off < kPiece ? bytes - off : kPiece, &bar);
     }
     if constexpr (ROT) {
-        prefetch_l2_cta(x, K * 2);
+        prefetch_l2_grid(x, K * 2);
     } else {
-        prefetch_l2_cta(q, K);
-        if (tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(s_a));
+        prefetch_l2_grid(q, K);
+        if (blockIdx.x == gridDim.x - 1 && tid == 0) asm volatile("prefetch.global.L2 [%0];" ::"l"(s_a));
     }
     griddep_launch_dependents();
     griddep_wait();
