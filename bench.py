@@ -59,14 +59,14 @@ def peaks():
 # as null.  `scale` converts the captured launch to the benchmarked one when the shapes differ
 # (traffic grows in proportion to the weights processed).
 PROFILED_TRAFFIC = {
-    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="ac7b33485df99f62", bytes=4231168 + 0,
+    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="b6667d172c58909a", bytes=4231168 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
-    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="5a0db57999d1fc9e",
-                    bytes=19753728 + 1263104, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
-    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="11e0d18d1b6121e0", bytes=14854144 + 0,
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="1cb8a9e37443764c",
+                    bytes=19752192 + 1284864, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="312551652af22a8e", bytes=14854144 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
-    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="d77053b1a3d2c13a",
-                    bytes=67137024 + 690688, scale=14336 * 4096 / (4096 * 4096),
+    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="c1010d5aaaed526a",
+                    bytes=67147264 + 1109760, scale=14336 * 4096 / (4096 * 4096),
                     profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
 }
 
