@@ -533,6 +533,9 @@ def run_offline(args, rank, world):
     t_qw = time_region(torch, lambda i: L.qift_quantize_weights(qg._ptr(rb), n_out, n_in, 0, 100, 0.2, 1.0,
                                                                 qg._ptr(codes), qg._ptr(scales), None,
                                                                 qg._stream(None)), 3) / 3
+    t_fused = time_region(torch, lambda i: qg._check(L.qift_rotate_quantize_weights(
+        qg._ptr(wbig), n_out, n_in, synth.MODEL_8B_BLOCK, 0, 100, 0.2, 1.0, qg._ptr(codes), qg._ptr(scales), None,
+        qg._stream(None)), "qift_rotate_quantize_weights"), 3) / 3
     evals = n_out * n_in * 100 / t_qw
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
     peak = alu_peak_evals(sm_mhz)
@@ -558,7 +561,9 @@ def run_offline(args, rank, world):
         "stages": {"a1_rotate_weights": {"ms": t_rot * 1e3, "GB/s": rot_b / t_rot / 1e9,
                                          "frac_hbm": rot_b / t_rot / 1e9 / peaks()["hbm_gbs"], "bound": "hbm"},
                    "a2_quantize_weights": {"ms": t_qw * 1e3, "candidate_evals_per_s": evals, "bound": "alu",
-                                           "frac_alu": evals / peak}},
+                                           "frac_alu": evals / peak},
+                   "a1a2_fused_rotate_quantize": {"ms": t_fused * 1e3, "two_calls_ms": (t_rot + t_qw) * 1e3,
+                                                  "entry": "qift_rotate_quantize_weights (one level set)"}},
     }
 
 

@@ -85,6 +85,20 @@ qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_i
                                   float* scales, double* row_mse, void* stream);
 
 /*
+ * qift_rotate_quantize_weights -- the offline pipeline in one pass: qift_rotate of the weights
+ * (fp32) followed by qift_quantize_weights, fused.  Abstract: "Hadamard-rotated quantization
+ * pipeline".  The rotation runs on each CTA's rows in shared memory with the operations and
+ * order of qift_rotate, so codes, scales and row_mse are bit-identical to the two calls; HBM sees
+ * one fp32 read of W and no rotated temporary.
+ *   w     : fp32 [n_out][n_in], the raw weights (not modified).
+ *   block : Hadamard block b as in qift_rotate (n_in % b == 0); 0 = w is already rotated.
+ *   other arguments as in qift_quantize_weights.
+ */
+qift_status qift_rotate_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int32_t block,
+                                         qift_levelset set, int32_t grid_points, double lo, double hi,
+                                         uint32_t* codes, float* scales, double* row_mse, void* stream);
+
+/*
  * qift_quantize_acts -- optional rotation + symmetric per-token INT4 quantization.
  * Abstract: the "A4" of rotated W2A4 inference.
  *   x      : fp16 (binary16 bits) [tokens][n_in], n_in % 16 == 0, n_in <= 32768.

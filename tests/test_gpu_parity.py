@@ -126,6 +126,35 @@ def test_quantize_weights_tiny_rows():
         assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
 
 
+# ------------------------------------------- fused offline pass: rotation + quantization
+@pytest.mark.parametrize("name", ["qift", "pot", "std"])
+@pytest.mark.parametrize("n_out,n_in,block", [(256, 512, 512), (300, 4096, 128), (37, 14336, 128), (9, 4096, 4096),
+                                              (5, 64, 16), (130, 1024, 2), (3, 32768, 4096)])
+def test_rotate_quantize_weights_fused(name, n_out, n_in, block):
+    # Same bits as the oracle's rotate-then-quantize and as the two library calls, for R = 4, 2
+    # and 1 rows per CTA, every block size class, and the largest row.
+    w = synth.weights(n_out, n_in, (n_in, block, 5))
+    codes, scales, mse, _ = oracle.quantize_weights(oracle.rotate_f32(w, block), name)
+    gw = dev(w)
+    gc, gs, gm = qg.qift_rotate_quantize_weights(gw, block, name)
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+    assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+    c2, s2, m2 = qg.qift_quantize_weights(qg.qift_rotate(gw, block), name)
+    assert torch.equal(gc, c2) and torch.equal(gs, s2) and torch.equal(gm, m2)
+    assert np.array_equal(host(gw), w)  # the raw weights are left as they were
+
+
+def test_rotate_quantize_weights_block0_and_bad_block():
+    w = synth.weights(4, 256, (6,))
+    gc, gs, gm = qg.qift_rotate_quantize_weights(dev(w), 0, "qift")
+    codes, scales, mse, _ = oracle.quantize_weights(w, "qift")
+    assert np.array_equal(codes_u32(gc), codes) and np.array_equal(host(gs), scales)
+    for bad in (3, 512, 8192):
+        with pytest.raises(qg.QiftError):
+            qg.qift_rotate_quantize_weights(dev(w), bad, "qift")
+
+
 # -------------------------------------------------------------------- activation quantizer
 @pytest.mark.parametrize("block", [0, 16, 128, 512, 4096])
 @pytest.mark.parametrize("T,K", [(1, 4096), (3, 512), (16, 11008), (33, 4096)])

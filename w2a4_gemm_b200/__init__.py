@@ -44,6 +44,7 @@ def lib() -> C.CDLL:
         i64, i32, f64, vp = C.c_int64, C.c_int32, C.c_double, C.c_void_p
         L.qift_rotate.argtypes = [vp, vp, i32, i64, i64, i32, vp]
         L.qift_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
+        L.qift_rotate_quantize_weights.argtypes = [vp, i64, i64, i32, i32, i32, f64, f64, vp, vp, vp, vp]
         L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
         L.qift_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, i32, vp]
         L.qift_decode_linear.argtypes = [vp, i64, i64, i32, vp, vp, i32, i64, vp, i32, vp, vp, vp]
@@ -55,7 +56,8 @@ def lib() -> C.CDLL:
         L.qift_debug_set_pdl.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
-        for name in ("qift_rotate", "qift_quantize_weights", "qift_quantize_acts", "qift_linear", "qift_decode_linear",
+        for name in ("qift_rotate", "qift_quantize_weights", "qift_rotate_quantize_weights", "qift_quantize_acts",
+                     "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
                      "qift_debug_stall_next_one_token",
                      "qift_debug_set_linear_path", "qift_debug_set_pdl"):
@@ -125,6 +127,22 @@ def qift_quantize_weights(w_rot: torch.Tensor, levelset="qift", grid_points: int
     _check(lib().qift_quantize_weights(_ptr(w_rot), n_out, n_in, _set(levelset), grid_points, lo, hi,
                                        _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
            "qift_quantize_weights")
+    return codes, scales, mse
+
+
+def qift_rotate_quantize_weights(w: torch.Tensor, block: int, levelset="qift", grid_points: int = 100,
+                                 lo: float = 0.2, hi: float = 1.0, with_mse: bool = True, stream=None):
+    """Rotation (block b; 0 = none) + scale search + encode + pack in one pass over the raw
+    weights.  Same outputs, bit for bit, as ``qift_quantize_weights(qift_rotate(w, b))``."""
+    _cuda(w, "w", torch.float32)
+    n_out, n_in = w.shape
+    dev = w.device
+    codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
+    scales = torch.empty(n_out, dtype=torch.float32, device=dev)
+    mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
+    _check(lib().qift_rotate_quantize_weights(_ptr(w), n_out, n_in, block, _set(levelset), grid_points, lo, hi,
+                                              _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
+           "qift_rotate_quantize_weights")
     return codes, scales, mse
 
 

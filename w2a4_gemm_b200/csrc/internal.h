@@ -39,9 +39,11 @@ cudaError_t launch_rotate(const void* x, void* y, bool f16, int64_t rows, int64_
 cudaError_t launch_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int block, int8_t* q,
                                  float* scales, cudaStream_t s);
 
+// block > 0: w holds raw weights, rotated by W H_b^T in shared memory first (same bits as
+// qift_rotate), so the offline pipeline reads each weight once and writes no fp32 temporary.
 cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int set, int grid_points,
                                     double lo, double hi, uint32_t* codes, float* scales, double* row_mse,
-                                    cudaStream_t s);
+                                    cudaStream_t s, int block = 0);
 
 // Decode-size linear: HBM-streaming GEMV (CUDA-core dp4a).
 cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,

@@ -19,7 +19,7 @@
 
 #include <algorithm>
 
-#include "common.cuh"
+#include "fwht.cuh"
 #include "internal.h"
 
 namespace qift {
@@ -71,14 +71,85 @@ struct Encoder {
 constexpr int kQwMaxRows = 4;   // rows per CTA
 constexpr int kQwMaxG = 256;     // candidates per row (API limit)
 
+// Block Walsh-Hadamard of every length-2^logb segment of the staged rows, in place (the fused
+// offline rotation): stages h = 1, 2, ..., b/2 of (lo + hi, lo - hi) in fp32, then one
+// multiply by c -- the operations and the order of qift_rotate, so the rows come out the same
+// bits as W H_b^T.
+//
+// b <= 512: a segment lives in the registers of b/16 lanes of one warp (fwht_segment: register
+// and shuffle stages, no barrier).  Every lane of a warp runs each pass, lanes past the last
+// segment on zeros, so the shuffles always see the whole warp.
+template <int LOGB>
+__device__ __forceinline__ void fwht_rows_regs(float* ws, int n_seg, float c) {
+    using S = FwhtShape<LOGB>;
+    static_assert(S::W == 1, "one warp per segment at most");
+    constexpr int SPW = 32 / S::TPS;  // segments per warp pass
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int ts = lane & (S::TPS - 1), sl = lane / S::TPS;
+    for (int base = warp * SPW; base < n_seg; base += nwarps * SPW) {  // warp-uniform
+        const int seg = base + sl;
+        const bool active = seg < n_seg;
+        float v[S::E];
+        if (active) {
+            load_contig<S::E>(ws + (size_t)seg * S::B + ts * S::E, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < S::E; ++i) v[i] = 0.0f;
+        }
+        float out[1][S::R];
+        fwht_segment<LOGB>(v, ts, lane, c, nullptr, out);
+        if (active) store_contig<S::R>(ws + (size_t)seg * S::B + ts * S::R, out[0]);
+    }
+}
+
+// b > 512: one barrier per stage over the whole CTA.
+__device__ __forceinline__ void fwht_rows_smem(float* ws, int rows, int K, int logb, float c) {
+    const int pairs = rows * K / 2;
+    for (int st = 0; st < logb; ++st) {
+        const int h = 1 << st;
+        const bool last = st == logb - 1;
+        for (int p = threadIdx.x; p < pairs; p += blockDim.x) {
+            const int lo = ((p >> st) << (st + 1)) | (p & (h - 1));  // pairs never cross a block
+            const float a = ws[lo], b = ws[lo + h];
+            float u = __fadd_rn(a, b), v = __fsub_rn(a, b);
+            if (last) {
+                u = __fmul_rn(u, c);
+                v = __fmul_rn(v, c);
+            }
+            ws[lo] = u;
+            ws[lo + h] = v;
+        }
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ void fwht_rows_in_smem(float* ws, int rows, int K, int logb, float c) {
+    const int n_seg = (rows * K) >> logb;
+    switch (logb) {
+        case 1: fwht_rows_regs<1>(ws, n_seg, c); break;
+        case 2: fwht_rows_regs<2>(ws, n_seg, c); break;
+        case 3: fwht_rows_regs<3>(ws, n_seg, c); break;
+        case 4: fwht_rows_regs<4>(ws, n_seg, c); break;
+        case 5: fwht_rows_regs<5>(ws, n_seg, c); break;
+        case 6: fwht_rows_regs<6>(ws, n_seg, c); break;
+        case 7: fwht_rows_regs<7>(ws, n_seg, c); break;
+        case 8: fwht_rows_regs<8>(ws, n_seg, c); break;
+        case 9: fwht_rows_regs<9>(ws, n_seg, c); break;
+        default: fwht_rows_smem(ws, rows, K, logb, c); return;
+    }
+    __syncthreads();
+}
+
 // One CTA owns R <= 4 output rows, staged together in shared memory, so that R x G (row,
 // candidate) pairs -- one per thread -- fill whole warps (G = 100 alone leaves a 128-thread CTA's
 // last warp with 4 busy lanes, and the bottleneck, the conversion unit, is paid per warp).
-template <int SET>
+// ROT: the rows are raw weights, rotated here first by 2^logb-point blocks (a1 and a2 in one
+// pass).
+template <int SET, bool ROT>
 __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __restrict__ w, int64_t n_out, int64_t K,
                                                              int R, int G, double lo, double hi,
                                                              uint32_t* __restrict__ codes, float* __restrict__ scales,
-                                                             double* __restrict__ row_mse) {
+                                                             double* __restrict__ row_mse, int logb, float c) {
     extern __shared__ __align__(16) float ws[];  // R rows of K floats
     __shared__ float cand[kQwMaxRows * kQwMaxG];
     __shared__ double mse[kQwMaxRows * kQwMaxG];
@@ -88,7 +159,16 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
     const int64_t row0 = (int64_t)blockIdx.x * R;
     const int rows = (int)min((int64_t)R, n_out - row0);
 
-    // Stage the rows and find each row's max |w|.
+    // Stage the rows (rotating them when asked) and find each row's max |w|.
+    if constexpr (ROT) {
+        for (int r = 0; r < rows; ++r) {
+            const float* wr = w + (row0 + r) * K;
+            for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4)
+                *reinterpret_cast<float4*>(ws + r * K + i) = *reinterpret_cast<const float4*>(wr + i);
+        }
+        __syncthreads();
+        fwht_rows_in_smem(ws, rows, (int)K, logb, c);
+    }
     float m[kQwMaxRows];
 #pragma unroll
     for (int r = 0; r < kQwMaxRows; ++r) {
@@ -96,8 +176,13 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
         if (r < rows) {
             const float* wr = w + (row0 + r) * K;
             for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4) {
-                const float4 v = *reinterpret_cast<const float4*>(wr + i);
-                *reinterpret_cast<float4*>(ws + r * K + i) = v;
+                float4 v;
+                if constexpr (ROT) {
+                    v = *reinterpret_cast<const float4*>(ws + r * K + i);
+                } else {
+                    v = *reinterpret_cast<const float4*>(wr + i);
+                    *reinterpret_cast<float4*>(ws + r * K + i) = v;
+                }
                 m[r] = fmaxf(m[r], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
             }
         }
@@ -178,28 +263,36 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
 
 template <int SET>
 static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
-                             uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
+                             uint32_t* codes, float* scales, double* row_mse, int block, cudaStream_t s) {
     // As many rows per CTA as fit in ~100 KB of shared memory (so several CTAs share an SM).
     int R = (int)std::min<int64_t>(kQwMaxRows, std::max<int64_t>(1, (100 * 1024) / (n_in * 4)));
     const int threads = std::max(128, std::min(1024, (R * G + 31) / 32 * 32));
     const size_t smem = (size_t)R * n_in * sizeof(float);
-    {
-        const cudaError_t e = ensure_smem(quant_weights_kernel<SET>, smem);
-        if (e != cudaSuccess) return e;
-    }
     const int64_t grid = (n_out + R - 1) / R;
-    quant_weights_kernel<SET><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes, scales,
-                                                                    row_mse);
+    if (block) {
+        const cudaError_t e = ensure_smem(quant_weights_kernel<SET, true>, smem);
+        if (e != cudaSuccess) return e;
+        // Normalisation constant as in qift_rotate: binary64 1/sqrt(b) rounded once to binary32.
+        const float c = (float)(1.0 / sqrt((double)block));
+        quant_weights_kernel<SET, true><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes,
+                                                                              scales, row_mse, ilog2(block), c);
+        return cudaGetLastError();
+    }
+    const cudaError_t e = ensure_smem(quant_weights_kernel<SET, false>, smem);
+    if (e != cudaSuccess) return e;
+    quant_weights_kernel<SET, false><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes,
+                                                                           scales, row_mse, 0, 1.0f);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int set, int G, double lo,
-                                    double hi, uint32_t* codes, float* scales, double* row_mse, cudaStream_t s) {
+                                    double hi, uint32_t* codes, float* scales, double* row_mse, cudaStream_t s,
+                                    int block) {
     if (n_out == 0) return cudaSuccess;
     switch (set) {
-        case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
-        case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
-        case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, s);
+        case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
+        case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
+        case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
         default: return cudaErrorInvalidValue;
     }
 }
