@@ -65,8 +65,8 @@ PROFILED_TRAFFIC = {
                     bytes=19752192 + 1284864, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
     "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="312551652af22a8e", bytes=14854144 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
-    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="c1010d5aaaed526a",
-                    bytes=67147264 + 1109760, scale=14336 * 4096 / (4096 * 4096),
+    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="cb68d6cdb915937a",
+                    bytes=67147008 + 1017088, scale=14336 * 4096 / (4096 * 4096),
                     profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
 }
 
