@@ -42,8 +42,12 @@ def lib():
         L.qo_unpack_codes.argtypes = [vp, i64, i64, vp]
         L.qo_quantize_acts.argtypes = [vp, i64, i64, vp, vp]
         L.qo_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, vp]
+        L.qo_pack_int4.argtypes = [vp, i64, vp]
+        L.qo_unpack_int4.argtypes = [vp, i64, vp]
+        L.qo_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp]
         for name in ("qo_fwht_f64", "qo_rotate_f32", "qo_candidate_scales", "qo_quantize_weights",
-                     "qo_unpack_codes", "qo_quantize_acts", "qo_linear"):
+                     "qo_unpack_codes", "qo_quantize_acts", "qo_linear", "qo_pack_int4", "qo_unpack_int4",
+                     "qo_dequantize_kv"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -135,6 +139,42 @@ def quantize_acts(x: np.ndarray, block: int = 0):
     s = np.zeros(T, dtype=np.float32)
     _check(lib().qo_quantize_acts(_ptr(xf), T, K, _ptr(q), _ptr(s)), "quantize_acts")
     return q, s, xr
+
+
+# -------------------------------------------------------------------------------------- KV4
+def pack_int4(q: np.ndarray) -> np.ndarray:
+    """int8 [..., n] in [-8, 7] -> uint8 [..., n/2]: two's-complement nibbles, lower index low."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    out = np.zeros(q.shape[:-1] + (q.shape[-1] // 2,), dtype=np.uint8)
+    _check(lib().qo_pack_int4(_ptr(q), q.size, _ptr(out)), "pack_int4")
+    return out
+
+
+def unpack_int4(p: np.ndarray) -> np.ndarray:
+    p = np.ascontiguousarray(p, dtype=np.uint8)
+    out = np.zeros(p.shape[:-1] + (p.shape[-1] * 2,), dtype=np.int8)
+    _check(lib().qo_unpack_int4(_ptr(p), out.size, _ptr(out)), "unpack_int4")
+    return out
+
+
+def quantize_kv(x: np.ndarray, block: int):
+    """KV4: rotate by ``block`` (0 = none), per-token INT4, two codes per byte.
+
+    ``x`` is binary16 ``[T, n]``.  Returns ``(packed uint8 [T, n/2], s f32 [T])``.
+    """
+    q, s, _ = quantize_acts(x, block)
+    return pack_int4(q), s
+
+
+def dequantize_kv(packed: np.ndarray, scales: np.ndarray, block: int) -> np.ndarray:
+    """Inverse of ``quantize_kv`` up to the quantization error: (float)q * s in binary32, the
+    inverse rotation in binary32, one rounding to binary16.  Returns float16 ``[T, n]``."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    T, n = packed.shape[0], packed.shape[1] * 2
+    out = np.zeros((T, n), dtype=np.float32)
+    _check(lib().qo_dequantize_kv(_ptr(packed), _ptr(scales), T, n, block, _ptr(out)), "dequantize_kv")
+    return out.astype(np.float16)
 
 
 # ---------------------------------------------------------------------------------- linear

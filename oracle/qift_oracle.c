@@ -290,6 +290,50 @@ int qo_quantize_acts(const float* x, int64_t tokens, int64_t n_in, int8_t* q, fl
 }
 
 /* ---------------------------------------------------------------------------------------
+ * KV4 (the title's "Rotated W2A4/KV4 LLM Inference"): keys and values kept in 4 bits.  The page
+ * gives no scheme; the reading used here is the activation path's -- the K or V row of a token
+ * is Hadamard-rotated by blocks of the head dimension and quantized to symmetric per-token INT4
+ * (qo_quantize_acts) -- with the codes stored two per byte.
+ *   pack:   byte j of a row = (q[2j] & 0xF) | ((q[2j+1] & 0xF) << 4)  (two's-complement nibbles,
+ *           the lower index in the low nibble);
+ *   unpack: the inverse, sign-extending each nibble;
+ *   dequantize: x = (float)q * s (one binary32 multiply), then the inverse rotation, which for
+ *           the normalised Sylvester matrix is the rotation itself (H/sqrt(b) is symmetric and
+ *           orthogonal): qo_rotate_f32's stages and final multiply.  The caller rounds to fp16.
+ * ------------------------------------------------------------------------------------- */
+int qo_pack_int4(const int8_t* q, int64_t n, uint8_t* out) {
+    if (!q || !out || n < 0 || (n & 1)) return -1;
+    for (int64_t j = 0; j < n / 2; ++j)
+        out[j] = (uint8_t)(((uint8_t)q[2 * j] & 0xFu) | (((uint8_t)q[2 * j + 1] & 0xFu) << 4));
+    return 0;
+}
+
+int qo_unpack_int4(const uint8_t* p, int64_t n, int8_t* q) {
+    if (!p || !q || n < 0 || (n & 1)) return -1;
+    for (int64_t j = 0; j < n / 2; ++j) {
+        const int lo = p[j] & 0xF, hi = p[j] >> 4;
+        q[2 * j] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+        q[2 * j + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+    }
+    return 0;
+}
+
+int qo_dequantize_kv(const uint8_t* packed, const float* scales, int64_t tokens, int64_t n, int32_t b,
+                     float* out) {
+    if (!packed || !scales || !out || tokens < 0 || n <= 0 || (n & 1)) return -1;
+    if (b != 0 && (!is_pow2(b) || (n % b) != 0)) return -1;
+    for (int64_t t = 0; t < tokens; ++t) {
+        int8_t* q = (int8_t*)malloc((size_t)n);
+        if (!q) return -2;
+        qo_unpack_int4(packed + t * (n / 2), n, q);
+        for (int64_t k = 0; k < n; ++k) out[t * n + k] = (float)q[k] * scales[t];
+        free(q);
+    }
+    if (b != 0) return qo_rotate_f32(out, tokens, n, b);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------------
  * W2A4 linear (Abstract: "sign-and-shift decoded weight application").
  *   acc[t][n] = sum_k q[t][k] * L(code[n][k])   (exact integer arithmetic, int64 here;
  *                                                 the result must fit int32)
