@@ -114,6 +114,25 @@ qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int3
                                float* scales, void* stream);
 
 /*
+ * qift_quantize_kv / qift_dequantize_kv -- KV4: keys and values kept in 4 bits (the title's
+ * "Rotated W2A4/KV4 LLM Inference").  The pages give no KV scheme; this one is the activation
+ * path's: each token's K or V row is rotated by Hadamard blocks of `block` (the head dimension,
+ * typically) and quantized to symmetric per-token INT4 exactly as qift_quantize_acts does, then
+ * stored as two's-complement nibbles, two per byte, the lower index in the low nibble.
+ *   x       : fp16 [tokens][n], n % 16 == 0, n <= 32768 (quantize) / 16384 (dequantize).
+ *   block   : 0 = no rotation; else a power of two in [2, 4096] dividing n.
+ *   packed  : u8 [tokens][n/2], 16-byte aligned.   scales: fp32 [tokens] (s = m / 7).
+ *   out     : fp16 [tokens][n]: (float)q * s in binary32, rotated back (H_b / sqrt(b) is its own
+ *             inverse) with qift_rotate's stages, rounded once to nearest even.
+ * Both are programmatic dependents of the previous kernel on `stream` that read their inputs
+ * only after it has finished.
+ */
+qift_status qift_quantize_kv(const void* x, int64_t tokens, int64_t n, int32_t block, uint8_t* packed,
+                             float* scales, void* stream);
+qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64_t tokens, int64_t n,
+                               int32_t block, void* out, void* stream);
+
+/*
  * qift_linear -- fused W2A4 linear: y[t][n] = ((float)acc[t][n] * w_scale[n]) * act_scale[t],
  * acc[t][n] = sum_k q_act[t][k] * level(code[n][k]) in int32.
  * Abstract: "sign-and-shift decoded weight application" of the fixed 2-bit levels.

@@ -88,6 +88,17 @@ def test_quantize_weights_parity(name, n_out, n_in, block):
     assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
 
 
+@pytest.mark.parametrize("n_in", [2560, 2816, 3072])
+def test_quantize_weights_static_plus_dynamic_smem_past_48k(n_in):
+    # Four rows of 2560..3072 inputs ask for 40..48 KB of dynamic shared memory; with the
+    # kernel's static buffers the total passes the default 48 KB limit.
+    w = oracle.rotate_f32(synth.weights(9, n_in, (n_in, 11)), 128)
+    codes, scales, mse, _ = oracle.quantize_weights(w, "qift")
+    gc, gs, gm = qg.qift_quantize_weights(dev(w), "qift")
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+
+
 def test_quantize_weights_edge_rows():
     # all-zero row, a single huge outlier, -0.0 entries, exact midpoints, constant row
     K = 64
@@ -153,6 +164,35 @@ def test_rotate_quantize_weights_block0_and_bad_block():
     for bad in (3, 512, 8192):
         with pytest.raises(qg.QiftError):
             qg.qift_rotate_quantize_weights(dev(w), bad, "qift")
+
+
+# ------------------------------------------------------------------- KV4 (packed INT4 K/V)
+@pytest.mark.parametrize("T,n,block", [(1, 128, 128), (7, 1024, 128), (300, 4096, 128), (16, 4096, 4096),
+                                       (5, 64, 0), (33, 8192, 64), (2, 16384, 128), (3, 1024, 1024)])
+def test_kv4_quantize_dequantize_match_oracle(T, n, block):
+    x = synth.activations(T, n, (T, n, block), n_outliers=synth.outlier_count(n))
+    x[0, : n // 2] = 0  # a half-zero token beside ordinary ones
+    packed, s = oracle.quantize_kv(x, block)
+    gp, gs = qg.qift_quantize_kv(dev(x), block)
+    assert np.array_equal(host(gp), packed)
+    assert np.array_equal(host(gs).view(np.uint32), s.view(np.uint32))
+    ref = oracle.dequantize_kv(packed, s, block)
+    gx = qg.qift_dequantize_kv(gp, gs, block)
+    assert np.array_equal(host(gx).view(np.uint16), ref.view(np.uint16))
+
+
+def test_kv4_zero_token_and_bad_arguments():
+    x = np.zeros((2, 256), np.float16)
+    gp, gs = qg.qift_quantize_kv(dev(x), 128)
+    assert int(gp.abs().sum() if gp.dtype != torch.uint8 else gp.sum()) == 0 and float(gs.abs().sum()) == 0.0
+    assert float(qg.qift_dequantize_kv(gp, gs, 128).abs().sum()) == 0.0
+    with pytest.raises(qg.QiftError):
+        qg.qift_quantize_kv(dev(np.zeros((2, 200), np.float16)), 0)      # n % 16
+    with pytest.raises(qg.QiftError):
+        qg.qift_quantize_kv(dev(x), 96)                                   # not a power of two
+    with pytest.raises(qg.QiftError):
+        qg.qift_dequantize_kv(torch.zeros((1, 16384), dtype=torch.uint8, device="cuda"),
+                              torch.ones(1, device="cuda"), 128)          # n = 32768 > 16384
 
 
 # -------------------------------------------------------------------- activation quantizer

@@ -46,6 +46,8 @@ def lib() -> C.CDLL:
         L.qift_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
         L.qift_rotate_quantize_weights.argtypes = [vp, i64, i64, i32, i32, i32, f64, f64, vp, vp, vp, vp]
         L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+        L.qift_quantize_kv.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+        L.qift_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp, vp]
         L.qift_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, i32, vp]
         L.qift_decode_linear.argtypes = [vp, i64, i64, i32, vp, vp, i32, i64, vp, i32, vp, vp, vp]
         L.qift_device_error.argtypes = [vp, C.POINTER(i32)]
@@ -57,6 +59,7 @@ def lib() -> C.CDLL:
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_rotate_quantize_weights", "qift_quantize_acts",
+                     "qift_quantize_kv", "qift_dequantize_kv",
                      "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
                      "qift_debug_stall_next_one_token",
@@ -156,6 +159,29 @@ def qift_quantize_acts(x: torch.Tensor, block: int = 0, out_q: torch.Tensor | No
         _cuda(out_scales, "out_scales", torch.float32)
     _check(lib().qift_quantize_acts(_ptr(x), T, K, block, _ptr(q), _ptr(s), _stream(stream)), "qift_quantize_acts")
     return q, s
+
+
+def qift_quantize_kv(x: torch.Tensor, block: int, stream=None):
+    """KV4: rotation by ``block`` + per-token INT4, two codes per byte.
+    Returns ``(packed uint8 [T, n/2], scales f32 [T])``."""
+    _cuda(x, "x", torch.float16)
+    T, n = x.shape
+    packed = torch.empty((T, n // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(T, dtype=torch.float32, device=x.device)
+    _check(lib().qift_quantize_kv(_ptr(x), T, n, block, _ptr(packed), _ptr(scales), _stream(stream)),
+           "qift_quantize_kv")
+    return packed, scales
+
+
+def qift_dequantize_kv(packed: torch.Tensor, scales: torch.Tensor, block: int, stream=None) -> torch.Tensor:
+    """Inverse of ``qift_quantize_kv`` up to the quantization error: fp16 [T, n]."""
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.float32)
+    T, n2 = packed.shape
+    out = torch.empty((T, 2 * n2), dtype=torch.float16, device=packed.device)
+    _check(lib().qift_dequantize_kv(_ptr(packed), _ptr(scales), T, 2 * n2, block, _ptr(out), _stream(stream)),
+           "qift_dequantize_kv")
+    return out
 
 
 def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w_scale: torch.Tensor,

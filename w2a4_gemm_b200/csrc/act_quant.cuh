@@ -54,11 +54,13 @@ __host__ __device__ constexpr size_t act_tbuf_bytes() {
     }
 }
 
-// Rotate one token (K fp16 values at xt, K % 16 == 0) into xs as fp16 and return max |x'|.
-// LOGB == 0: the token is already rotated (copied as is).  `red` holds kActThreads/32 floats.
-template <int LOGB, typename Bar = CtaSync>
-__device__ __forceinline__ float rotate_token_f16(const __half* __restrict__ xt, int64_t K, float c, __half* xs,
+// Rotate one token (K values at xt, fp16 or fp32, K % 16 == 0) into xs as fp16 and return
+// max |x'|.  LOGB == 0: the token is already rotated (fp16 input only, copied as is).  `red`
+// holds kActThreads/32 floats.
+template <int LOGB, typename Bar = CtaSync, typename InT = __half>
+__device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, int64_t K, float c, __half* xs,
                                                   float* tbuf, float* red) {
+    static_assert(LOGB > 0 || sizeof(InT) == 2, "the copy path takes fp16 input");
     const int tid = threadIdx.x, lane = tid & 31;
     float amax = 0.0f;
     if constexpr (LOGB == 0) {
@@ -164,6 +166,14 @@ __device__ __forceinline__ uint4 quant16(const __half* xs16, float inv) {
         packed[w] = word;
     }
     return make_uint4(packed[0], packed[1], packed[2], packed[3]);
+}
+
+// Sixteen INT4 codes (int8 bytes, from quant16) -> eight bytes of two's-complement nibbles, the
+// lower index in the low nibble.  Per word: keep the low nibbles, fold byte 2j+1's nibble onto
+// byte 2j, then one byte permute gathers bytes 0 and 2 of two words.
+__device__ __forceinline__ uint2 pack_int4_16(uint4 v) {
+    const uint32_t a = v.x & 0x0F0F0F0Fu, b = v.y & 0x0F0F0F0Fu, c = v.z & 0x0F0F0F0Fu, d = v.w & 0x0F0F0F0Fu;
+    return make_uint2(prmt(a | (a >> 4), b | (b >> 4), 0x6420u), prmt(c | (c >> 4), d | (d >> 4), 0x6420u));
 }
 
 }  // namespace qift

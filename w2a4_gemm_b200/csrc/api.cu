@@ -114,6 +114,31 @@ qift_status qift_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int3
         qift::launch_quantize_acts(x, tokens, n_in, block, q, scales, static_cast<cudaStream_t>(stream)));
 }
 
+qift_status qift_quantize_kv(const void* x, int64_t tokens, int64_t n, int32_t block, uint8_t* packed,
+                             float* scales, void* stream) {
+    if (tokens < 0 || n <= 0 || n % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (block != 0 && (!valid_block(block) || n % block != 0)) return QIFT_ERR_INVALID_ARG;
+    if (n > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (tokens == 0) return QIFT_OK;
+    if (!x || !packed || !scales || !aligned16(x) || !aligned16(packed) || !aligned4(scales))
+        return QIFT_ERR_INVALID_ARG;
+    if (tokens > 0x7fffffff) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(qift::launch_quantize_kv(x, tokens, n, block, packed, scales, static_cast<cudaStream_t>(stream)));
+}
+
+qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64_t tokens, int64_t n, int32_t block,
+                               void* out, void* stream) {
+    if (tokens < 0 || n <= 0 || n % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (block != 0 && (!valid_block(block) || n % block != 0)) return QIFT_ERR_INVALID_ARG;
+    if (n > 16384) return QIFT_ERR_UNSUPPORTED;
+    if (tokens == 0) return QIFT_OK;
+    if (!packed || !scales || !out || !aligned16(packed) || !aligned16(out) || !aligned4(scales))
+        return QIFT_ERR_INVALID_ARG;
+    if (tokens > 0x7fffffff) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(
+        qift::launch_dequantize_kv(packed, scales, tokens, n, block, out, static_cast<cudaStream_t>(stream)));
+}
+
 qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint32_t* codes, const float* w_scale,
                         qift_levelset set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, qift_dtype out_dt,
                         void* stream) {

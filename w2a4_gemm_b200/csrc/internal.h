@@ -27,9 +27,11 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // including ones captured into CUDA graphs -- do not repeat the attribute call.
 cudaError_t ensure_smem_ptr(const void* kernel, size_t bytes);
 
+// Called for any dynamic size: the default 48 KB limit covers static plus dynamic shared memory,
+// so a kernel with static buffers can pass it with less than 48 KB requested.
 template <typename Kernel>
 inline cudaError_t ensure_smem(Kernel kernel, size_t bytes) {
-    if (bytes <= 48 * 1024) return cudaSuccess;
+    if (bytes == 0) return cudaSuccess;
     return ensure_smem_ptr(reinterpret_cast<const void*>(kernel), bytes);
 }
 
@@ -38,6 +40,12 @@ cudaError_t launch_rotate(const void* x, void* y, bool f16, int64_t rows, int64_
 
 cudaError_t launch_quantize_acts(const void* x, int64_t tokens, int64_t n_in, int block, int8_t* q,
                                  float* scales, cudaStream_t s);
+
+// KV4: the activation quantizer with the codes packed two per byte, and its inverse.
+cudaError_t launch_quantize_kv(const void* x, int64_t tokens, int64_t n, int block, uint8_t* packed, float* scales,
+                               cudaStream_t s);
+cudaError_t launch_dequantize_kv(const uint8_t* packed, const float* scales, int64_t tokens, int64_t n, int block,
+                                 void* out, cudaStream_t s);
 
 // block > 0: w holds raw weights, rotated by W H_b^T in shared memory first (same bits as
 // qift_rotate), so the offline pipeline reads each weight once and writes no fp32 temporary.
