@@ -54,6 +54,29 @@ __host__ __device__ constexpr size_t act_tbuf_bytes() {
     }
 }
 
+// R contiguous fp16 values (R even) from R/2 packed pairs.
+template <int R>
+__device__ __forceinline__ void store_half2s(__half* __restrict__ p, const __half2 (&h)[R / 2]) {
+    if constexpr (R >= 8) {
+#pragma unroll
+        for (int i = 0; i < R / 2; i += 4) {
+            uint4 t;
+            t.x = *reinterpret_cast<const uint32_t*>(&h[i]);
+            t.y = *reinterpret_cast<const uint32_t*>(&h[i + 1]);
+            t.z = *reinterpret_cast<const uint32_t*>(&h[i + 2]);
+            t.w = *reinterpret_cast<const uint32_t*>(&h[i + 3]);
+            *reinterpret_cast<uint4*>(p + 2 * i) = t;
+        }
+    } else if constexpr (R == 4) {
+        uint2 t;
+        t.x = *reinterpret_cast<const uint32_t*>(&h[0]);
+        t.y = *reinterpret_cast<const uint32_t*>(&h[1]);
+        *reinterpret_cast<uint2*>(p) = t;
+    } else {
+        *reinterpret_cast<__half2*>(p) = h[0];
+    }
+}
+
 // Rotate one token (K values at xt, fp16 or fp32, K % 16 == 0) into xs as fp16 and return
 // max |x'|.  LOGB == 0: the token is already rotated (fp16 input only, copied as is).  `red`
 // holds kActThreads/32 floats.
@@ -62,17 +85,15 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
                                                   float* tbuf, float* red) {
     static_assert(LOGB > 0 || sizeof(InT) == 2, "the copy path takes fp16 input");
     const int tid = threadIdx.x, lane = tid & 31;
-    float amax = 0.0f;
+    // max |x'| is taken on the fp16 values themselves, two at a time: a max does not round.
+    __half2 amax2 = __float2half2_rn(0.0f);
     if constexpr (LOGB == 0) {
         for (int64_t i = (int64_t)tid * 8; i < K; i += kActThreads * 8) {
             const uint4 t = *reinterpret_cast<const uint4*>(xt + i);
             *reinterpret_cast<uint4*>(xs + i) = t;
             const __half2* h = reinterpret_cast<const __half2*>(&t);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __half22float2(h[j]);
-                amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
+            for (int j = 0; j < 4; ++j) amax2 = __hmax2(amax2, __habs2(h[j]));
         }
     } else if constexpr (LOGB == 12) {
         static_assert(kActThreads == 256, "one 16-value column per thread");
@@ -95,10 +116,11 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
             for (int i = 0; i < 16; ++i) v[i] = tbuf[tpad4096(tid + 256 * i)];
             reg_stages<16>(v);  // h = 256 .. 2048
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const __half h = __float2half_rn(__fmul_rn(v[i], c));
-                amax = fmaxf(amax, fabsf(__half2float(h)));
-                xs[seg * 4096 + tid + 256 * i] = h;
+            for (int i = 0; i < 16; i += 2) {
+                const __half2 h = __floats2half2_rn(__fmul_rn(v[i], c), __fmul_rn(v[i + 1], c));
+                amax2 = __hmax2(amax2, __habs2(h));
+                xs[seg * 4096 + tid + 256 * i] = __low2half(h);
+                xs[seg * 4096 + tid + 256 * (i + 1)] = __high2half(h);
             }
             Bar::sync();  // tbuf is reused by the next segment
         }
@@ -123,24 +145,29 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
             if (active) {
 #pragma unroll
                 for (int j = 0; j < S::W; ++j) {
-                    float hv[S::R];
+                    __half2 hv[S::R / 2];
 #pragma unroll
-                    for (int r = 0; r < S::R; ++r) {
-                        hv[r] = __half2float(__float2half_rn(out[j][r]));
-                        amax = fmaxf(amax, fabsf(hv[r]));
+                    for (int r = 0; r < S::R; r += 2) {
+                        hv[r / 2] = __floats2half2_rn(out[j][r], out[j][r + 1]);
+                        amax2 = __hmax2(amax2, __habs2(hv[r / 2]));
                     }
-                    store_contig<S::R>(xs + seg * S::B + ts * S::R + j * S::COL, hv);
+                    store_half2s<S::R>(xs + seg * S::B + ts * S::R + j * S::COL, hv);
                 }
             }
             if constexpr (S::W > 1) Bar::sync();  // tbuf is reused by the next pass
         }
     }
     Bar::sync();
-    return block_max<Bar>(amax, red);
+    const float2 a = __half22float2(amax2);
+    return block_max<Bar>(fmaxf(a.x, a.y), red);
 }
 
 // Sixteen fp16 values -> sixteen INT4 codes in int8 bytes, natural order:
 // clamp(rint_even(x * inv), -7, 7), one fp32 multiply per value.  inv = 7/m (IEEE division).
+// rint is the magic-number add on the fp32 pipe: t = x * inv + 1.5 * 2^23 is exact and its
+// low byte is the code in two's complement, so byte permutes gather the codes.  The clamp never
+// binds: |x| <= m and inv <= (7/m)(1 + 2^-24), so |x * inv| < 7.5 and the rounded value is at
+// most 7 in magnitude.
 __device__ __forceinline__ uint4 quant16(const __half* xs16, float inv) {
     const uint4 a = *reinterpret_cast<const uint4*>(xs16);
     const uint4 b = *reinterpret_cast<const uint4*>(xs16 + 8);
@@ -152,18 +179,11 @@ __device__ __forceinline__ uint4 quant16(const __half* xs16, float inv) {
         const __half2* h = w < 2 ? ha + 2 * w : hb + 2 * (w - 2);
         const float2 f0 = __half22float2(h[0]);
         const float2 f1 = __half22float2(h[1]);
-        const float f[4] = {f0.x, f0.y, f1.x, f1.y};
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            // rint (half to even) by the magic-number add, on the fp32 pipe instead of the
-            // conversion unit: exact for |t| < 2^22, and |x * 7/m| <= 7 (1 + 2^-23) here.
-            const float t = __fadd_rn(__fmul_rn(f[e], inv), 12582912.0f);
-            int v = __float_as_int(t) - 0x4B400000;
-            v = v > 7 ? 7 : (v < -7 ? -7 : v);
-            word |= (uint32_t)(v & 0xff) << (8 * e);
-        }
-        packed[w] = word;
+        const uint32_t t0 = __float_as_uint(__fadd_rn(__fmul_rn(f0.x, inv), 12582912.0f));
+        const uint32_t t1 = __float_as_uint(__fadd_rn(__fmul_rn(f0.y, inv), 12582912.0f));
+        const uint32_t t2 = __float_as_uint(__fadd_rn(__fmul_rn(f1.x, inv), 12582912.0f));
+        const uint32_t t3 = __float_as_uint(__fadd_rn(__fmul_rn(f1.y, inv), 12582912.0f));
+        packed[w] = prmt(prmt(t0, t1, 0x0040u), prmt(t2, t3, 0x0040u), 0x5410u);
     }
     return make_uint4(packed[0], packed[1], packed[2], packed[3]);
 }

@@ -47,17 +47,19 @@ __device__ __forceinline__ void reg_stages(float (&v)[E]) {
     }
 }
 
-// Butterflies across lanes: the lane without bit m holds u, the lane with it holds v.
+// Butterflies across lanes: the lane without bit m holds u, the lane with it holds v; the
+// lower lane keeps u + v, the upper one u - v.  Both are fma(sgn, own, partner) with sgn = +1
+// or -1: sgn * own is exact, so the one rounding gives the same bits as the add or subtract.
 template <int E, int LANE_BITS>
 __device__ __forceinline__ void lane_stages(float (&v)[E], int lane) {
 #pragma unroll
     for (int j = 0; j < LANE_BITS; ++j) {
         const int m = 1 << j;
-        const bool upper = (lane & m) != 0;
+        const float sgn = (lane & m) ? -1.0f : 1.0f;
 #pragma unroll
         for (int i = 0; i < E; ++i) {
             const float p = __shfl_xor_sync(0xffffffffu, v[i], m);
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+            v[i] = __fmaf_rn(sgn, v[i], p);
         }
     }
 }
