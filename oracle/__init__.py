@@ -42,12 +42,14 @@ def lib():
         L.qo_unpack_codes.argtypes = [vp, i64, i64, vp]
         L.qo_quantize_acts.argtypes = [vp, i64, i64, vp, vp]
         L.qo_linear.argtypes = [vp, vp, vp, vp, i32, i64, i64, i64, vp, vp]
+        L.qo_quantize_weights_w4.argtypes = [vp, i64, i64, i32, f64, f64, vp, vp, vp, vp]
+        L.qo_linear_w4.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
         L.qo_pack_int4.argtypes = [vp, i64, vp]
         L.qo_unpack_int4.argtypes = [vp, i64, vp]
         L.qo_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp]
         for name in ("qo_fwht_f64", "qo_rotate_f32", "qo_candidate_scales", "qo_quantize_weights",
                      "qo_unpack_codes", "qo_quantize_acts", "qo_linear", "qo_pack_int4", "qo_unpack_int4",
-                     "qo_dequantize_kv"):
+                     "qo_dequantize_kv", "qo_quantize_weights_w4", "qo_linear_w4"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -139,6 +141,50 @@ def quantize_acts(x: np.ndarray, block: int = 0):
     s = np.zeros(T, dtype=np.float32)
     _check(lib().qo_quantize_acts(_ptr(xf), T, K, _ptr(q), _ptr(s)), "quantize_acts")
     return q, s, xr
+
+
+# --------------------------------------------------------------------------------------- W4
+W4_LEVELS = np.arange(-7, 8, dtype=np.int32)
+
+
+def quantize_weights_w4(w_rot: np.ndarray, grid_points: int = 100, lo: float = 0.2, hi: float = 1.0):
+    """W4 per-channel scale search + nearest-level encode + pack (levels {-7..7} * s).
+
+    Returns ``(codes uint32 [N, K/8], scales f32 [N], row_mse f64 [N], best_k int32 [N])``;
+    the code of input k is ``level + 7`` at bits ``4*(k%8)`` of word ``k/8``.
+    """
+    w = np.ascontiguousarray(w_rot, dtype=np.float32)
+    n_out, n_in = w.shape
+    codes = np.zeros((n_out, n_in // 8), dtype=np.uint32)
+    scales = np.zeros(n_out, dtype=np.float32)
+    mse = np.zeros(n_out, dtype=np.float64)
+    best = np.zeros(n_out, dtype=np.int32)
+    _check(lib().qo_quantize_weights_w4(_ptr(w), n_out, n_in, grid_points, lo, hi, _ptr(codes), _ptr(scales),
+                                        _ptr(mse), _ptr(best)), "quantize_weights_w4")
+    return codes, scales, mse, best
+
+
+def unpack_w4(codes: np.ndarray, n_in: int) -> np.ndarray:
+    """uint32 [N, K/8] -> int8 levels [N, K] in [-7, 7]."""
+    c = np.ascontiguousarray(codes, dtype=np.uint32)
+    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
+    u = (c[:, :, None] >> shifts) & np.uint32(0xF)
+    return (u.reshape(c.shape[0], n_in).astype(np.int16) - 7).astype(np.int8)
+
+
+def linear_w4(q: np.ndarray, s_a: np.ndarray, codes: np.ndarray, s_w: np.ndarray, out_dtype=np.float32):
+    """W4A4 linear: int32 accumulators and the binary32 epilogue.  Returns ``(y, acc)``."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    T, K = q.shape
+    N = codes.shape[0]
+    assert codes.shape[1] * 8 == K
+    acc = np.zeros((T, N), dtype=np.int32)
+    y = np.zeros((T, N), dtype=np.float32)
+    _check(lib().qo_linear_w4(_ptr(q), _ptr(s_a), _ptr(codes), _ptr(s_w), T, N, K, _ptr(acc), _ptr(y)), "linear_w4")
+    return y.astype(out_dtype), acc
 
 
 # -------------------------------------------------------------------------------------- KV4

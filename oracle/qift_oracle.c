@@ -253,6 +253,107 @@ int qo_unpack_codes(const uint32_t* codes, int64_t n_out, int64_t n_in, uint8_t*
 }
 
 /* ---------------------------------------------------------------------------------------
+ * W4 weights (the Abstract's "L-layer mixed W2/W4": 4-bit layers beside the 2-bit ones).  The
+ * page gives no W4 scheme; the reading (R20) keeps this method's rule -- one scale per output
+ * channel, no zero point, the same MSE-searched candidate grid (R3, outer level 7) -- with the
+ * symmetric 4-bit integer levels {-7, ..., +7} * s.
+ *   encode: |w| against the midpoints (j + 0.5) s, j = 0..6, in binary64 (exact: a binary32
+ *           times j + 0.5 needs at most 28 bits); level magnitude = the number of midpoints
+ *           strictly below |w|, so a tie takes the smaller magnitude (R8); w >= 0 (and -0.0)
+ *           takes the positive side (R7);
+ *   error:  e = |w| - l, l = j * s in binary32, e * e in binary32, summed in binary64 in index
+ *           order (R9);
+ *   code:   u = level + 7 in [0, 14], eight per u32, the code of input k at bits 4*(k%8) .. +3,
+ *           least significant first (R21).  The stored scale is s itself.
+ * ------------------------------------------------------------------------------------- */
+static int32_t encode_w4(float w, float s) {
+    const double a = fabs((double)w), sd = (double)s;
+    int32_t j = 0;
+    while (j < 7 && a > ((double)j + 0.5) * sd) ++j;
+    return w >= 0.0f ? j : -j;
+}
+
+static float sq_err_w4(float w, float s, int32_t level) {
+    const float l = (float)(level < 0 ? -level : level) * s;
+    const float e = fabsf(w) - l;
+    return e * e;
+}
+
+int qo_quantize_weights_w4(const float* w, int64_t n_out, int64_t n_in, int32_t grid_points, double lo, double hi,
+                           uint32_t* codes, float* scales, double* row_mse, int32_t* best_k) {
+    if (!w || !codes || !scales || n_out < 0 || n_in <= 0 || (n_in % 8) != 0) return -1;
+    if (grid_points < 2 || grid_points > 4096) return -1;
+    const int64_t words = n_in / 8;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < n_out; ++n) {
+        const float* row = w + n * n_in;
+        float m = 0.0f;
+        for (int64_t k = 0; k < n_in; ++k) {
+            const float a = fabsf(row[k]);
+            if (a > m) m = a;
+        }
+        float* cand = (float*)malloc(sizeof(float) * (size_t)grid_points);
+        if (!cand) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        for (int32_t g = 0; g < grid_points; ++g) {  /* R3 with the outer level 7 */
+            const double f = lo + ((hi - lo) * (double)g) / (double)(grid_points - 1);
+            cand[g] = (float)((f * (double)m) / 7.0);
+        }
+        int32_t kbest = 0;
+        double best = 0.0;
+        for (int32_t g = 0; g < grid_points; ++g) {
+            const float s = cand[g];
+            double acc = 0.0;
+            for (int64_t k = 0; k < n_in; ++k) acc += (double)sq_err_w4(row[k], s, encode_w4(row[k], s));
+            if (g == 0 || acc < best) {
+                best = acc;
+                kbest = g;
+            }
+        }
+        const float s = cand[kbest];
+        free(cand);
+        uint32_t* out = codes + n * words;
+        for (int64_t j = 0; j < words; ++j) out[j] = 0u;
+        for (int64_t k = 0; k < n_in; ++k)
+            out[k / 8] |= (uint32_t)(encode_w4(row[k], s) + 7) << (4 * (k % 8));
+        scales[n] = s;
+        if (row_mse) row_mse[n] = best / (double)n_in;
+        if (best_k) best_k[n] = kbest;
+    }
+    return bad ? -2 : 0;
+}
+
+/* W4A4 linear: acc[t][n] = sum_k q[t][k] * (u(code) - 7) exactly (int64, must fit int32), then
+ * y = ((float)acc * s_w[n]) * s_a[t] (R13).  acc and y may be NULL. */
+int qo_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int64_t tokens,
+                 int64_t n_out, int64_t n_in, int32_t* acc_out, float* y) {
+    if (!q || !s_a || !codes || !s_w || tokens < 0 || n_out < 0 || n_in <= 0 || (n_in % 8) != 0) return -1;
+    const int64_t words = n_in / 8;
+    int overflow = 0;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t t = 0; t < tokens; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            int64_t sum = 0;
+            for (int64_t k = 0; k < n_in; ++k) {
+                const int32_t u = (int32_t)((codes[n * words + k / 8] >> (4 * (k % 8))) & 0xFu);
+                sum += (int64_t)q[t * n_in + k] * (int64_t)(u - 7);
+            }
+            if (sum > INT32_MAX || sum < INT32_MIN) {
+#pragma omp atomic write
+                overflow = 1;
+            }
+            if (acc_out) acc_out[t * n_out + n] = (int32_t)sum;
+            if (y) y[t * n_out + n] = ((float)sum * s_w[n]) * s_a[t];
+        }
+    }
+    return overflow ? -3 : 0;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Symmetric per-token INT4 activation quantization (the "A4" of W2A4 in the Abstract).
  * Input: the rotated activations after their single rounding to binary16, given here as
  * the binary32 values of those binary16 numbers.
