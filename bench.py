@@ -1,13 +1,16 @@
 """Benchmark of the Qift W2A4 linear path on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|decode16|prefill|single]
+                    [--workload decode|decode16|prefill|single|offline|decode_w4|decode16_w4]
 
 Workloads (synthetic, seeded; shapes of LLaMA linear modules):
   decode   (default) LLaMA-7B q_proj 4096x4096, 1 token, 4096-point Hadamard, Qift {+-1,+-3}
   decode16 LLaMA-3.1-8B MLP (gate/up 14336x4096, down 4096x14336), 16 tokens, 128-block, PoT
   prefill  LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008), 2048 tokens, 128-block, Qift
   single   one 256x512 linear, 8 tokens (parity case; timed for completeness)
+  decode_w4, decode16_w4
+           the decode and decode16 shapes with 4-bit weights ({-7..7} * s per channel), the
+           W4 layers of a mixed W2/W4 model: W4A4 linear on CUDA cores
   offline  offline quantization of a full 8B-shaped model (224 modules, 6.98 G weights):
            128-block rotation + per-row scale search + encode + pack for the Qift, PoT and
            standard level sets; reports weights/s and the reconstruction MSE of each set
@@ -89,12 +92,18 @@ def profiled_traffic(workload):
 def workload_def(name):
     from w2a4_gemm_b200 import synth
     return {"decode": synth.LLAMA7B_QPROJ_DECODE, "decode16": synth.LLAMA31_8B_MLP_DECODE16,
-            "prefill": synth.LLAMA7B_MLP_PREFILL, "single": synth.SINGLE_256x512}[name]
+            "prefill": synth.LLAMA7B_MLP_PREFILL, "single": synth.SINGLE_256x512,
+            "decode_w4": synth.LLAMA7B_QPROJ_DECODE_W4, "decode16_w4": synth.LLAMA31_8B_MLP_DECODE16_W4}[name]
 
 
-def linear_bytes(T, N, K, out_bytes):
+def code_bytes(N, K, levelset):
+    """Bytes of packed weight codes: 2 bits per weight, 4 for the 4-bit set."""
+    return N * K // 2 if levelset == "int4" else N * K // 4
+
+
+def linear_bytes(T, N, K, out_bytes, levelset="qift"):
     """Algorithmic HBM bytes of one qift_linear: codes + w scales + int8 acts + act scales + y."""
-    return N * K // 4 + 4 * N + T * K + 4 * T + T * N * out_bytes
+    return code_bytes(N, K, levelset) + 4 * N + T * K + 4 * T + T * N * out_bytes
 
 
 def acts_bytes(T, K):
@@ -264,11 +273,11 @@ def run_ours(args, rank, world):
     wl = workload_def(args.workload)
     pk = peaks()
     T = wl.tokens
-    wbytes = sum(l.n_out * l.n_in // 4 for l in wl.linears)
+    wbytes = sum(code_bytes(l.n_out, l.n_in, wl.levelset) for l in wl.linears)
     copies = max(1, min(64, int(np.ceil(3 * L2_BYTES / max(wbytes, 1))))) if T <= 16 else 1
     st = OursState(wl, torch, qg, copies)
     out_b = 2 if wl.out_dtype == "f16" else 4
-    step_bytes = sum(linear_bytes(T, l.n_out, l.n_in, out_b) for l in wl.linears)
+    step_bytes = sum(linear_bytes(T, l.n_out, l.n_in, out_b, wl.levelset) for l in wl.linears)
     step_ops = sum(2 * T * l.n_out * l.n_in for l in wl.linears)
     decode = T <= 16
 
@@ -300,7 +309,7 @@ def run_ours(args, rank, world):
                                                         L0["codes"][i % copies], L0["s_w"][i % copies], wl.levelset,
                                                         st.out_dt, out=L0["y"][i % copies]), reps) / reps
     t_fused = None
-    if T <= 4 and lin0.n_in % 64 == 0 and lin0.n_in <= 16384 and wl.levelset != "std":
+    if T <= 4 and lin0.n_in % 64 == 0 and lin0.n_in <= 16384 and wl.levelset in ("qift", "pot"):
         t_fused = time_region(torch, lambda i: qg.qift_decode_linear(L0["x"][i % copies], wl.a_block,
                                                                      L0["codes"][i % copies], L0["s_w"][i % copies],
                                                                      wl.levelset, st.out_dt, out=L0["y"][i % copies]),
@@ -311,7 +320,7 @@ def run_ours(args, rank, world):
     t_qw = time_region(torch, lambda i: qg.qift_quantize_weights(w_rot, wl.levelset, with_mse=False), 2) / 2
 
     N0, K0 = lin0.n_out, lin0.n_in
-    lin_b = linear_bytes(T, N0, K0, out_b)
+    lin_b = linear_bytes(T, N0, K0, out_b, wl.levelset)
     act_b = acts_bytes(T, K0)
     rot_b = 8 * N0 * K0
     stages = {
@@ -337,7 +346,7 @@ def run_ours(args, rank, world):
         unit = "GB/s"
         roof = {"bound": "hbm", "achieved": lin_b / t_lin / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": lin_b / t_lin / 1e9 / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload),
-                "kernel": "qift_linear (GEMV)",
+                "kernel": "qift_linear (W4A4 GEMV)" if wl.levelset == "int4" else "qift_linear (GEMV)",
                 "peak_source": pk["source"] + " copy bandwidth, burst"}
     else:
         value = world * step_ops * args.steps / secs / 1e12
@@ -437,7 +446,10 @@ def oracle_step_fn(wl, sample_tokens):
     seen = set()
     for lin in wl.linears:
         W = wl.w(lin)
-        codes, s_w, _, _ = oracle.quantize_weights(oracle.rotate_f32(W, wl.w_block), wl.levelset)
+        if wl.levelset == "int4":
+            codes, s_w, _, _ = oracle.quantize_weights_w4(oracle.rotate_f32(W, wl.w_block))
+        else:
+            codes, s_w, _, _ = oracle.quantize_weights(oracle.rotate_f32(W, wl.w_block), wl.levelset)
         x = wl.x(lin)[:sample_tokens]
         key = (lin.x_seed, lin.n_in)  # linears reading the same input share one quantization
         prepared.append((lin, codes, s_w, x, key not in seen))
@@ -448,7 +460,10 @@ def oracle_step_fn(wl, sample_tokens):
         for lin, codes, s_w, x, quant in prepared:
             if quant:
                 q, sa, _ = oracle.quantize_acts(x, wl.a_block)
-            oracle.linear(q, sa, codes, s_w, wl.levelset, np.float16)
+            if wl.levelset == "int4":
+                oracle.linear_w4(q, sa, codes, s_w, np.float16)
+            else:
+                oracle.linear(q, sa, codes, s_w, wl.levelset, np.float16)
 
     return step, prepared
 
@@ -466,7 +481,7 @@ def run_cpu(wl, budget_s, sample_tokens):
     secs = (time.perf_counter() - t0) / n
     T = sample_tokens
     out_b = 2
-    by = sum(linear_bytes(T, p[0].n_out, p[0].n_in, out_b) for p in prepared)
+    by = sum(linear_bytes(T, p[0].n_out, p[0].n_in, out_b, wl.levelset) for p in prepared)
     ops = sum(2 * T * p[0].n_out * p[0].n_in for p in prepared)
     return secs, by, ops, oracle.threads(), n
 
@@ -493,7 +508,7 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     secs = (time.perf_counter() - t0)
-    by = sum(linear_bytes(T, l.n_out, l.n_in, 2) for l, *_ in prepared)
+    by = sum(linear_bytes(T, l.n_out, l.n_in, 2, wl.levelset) for l, *_ in prepared)
     ops = sum(2 * T * l.n_out * l.n_in for l, *_ in prepared)
     val = (by if decode else ops) * args.steps / secs / (1e9 if decode else 1e12)
     unit = "GB/s" if decode else "TOPS"
@@ -635,7 +650,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single", "offline"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single", "offline", "decode_w4",
+                                           "decode16_w4"], default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))

@@ -67,7 +67,7 @@ def test_quantize_weights_validation(L):
     bad = q.QIFT_ERR_INVALID_ARG
     f = L.qift_quantize_weights
     assert f(FAKE, 4, 40, 0, 100, 0.2, 1.0, FAKE, FAKE, None, None) == bad    # n_in % 16
-    assert f(FAKE, 4, 64, 3, 100, 0.2, 1.0, FAKE, FAKE, None, None) == bad    # set
+    assert f(FAKE, 4, 64, 4, 100, 0.2, 1.0, FAKE, FAKE, None, None) == bad    # set
     assert f(FAKE, 4, 64, 0, 1, 0.2, 1.0, FAKE, FAKE, None, None) == bad      # grid
     assert f(FAKE, 4, 64, 0, 257, 0.2, 1.0, FAKE, FAKE, None, None) == bad
     assert f(FAKE, 4, 64, 0, 100, 0.0, 1.0, FAKE, FAKE, None, None) == bad    # lo
@@ -103,6 +103,11 @@ def test_linear_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 65536, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
     assert f(None, None, None, None, 0, 0, 8, 64, None, 1, None) == q.QIFT_OK                # no tokens
     assert f(None, None, None, None, 1, 3, 0, 64, None, 0, None) == q.QIFT_OK                # no outputs
+    # 4-bit weights (set 3): 1..16 tokens, n_in a multiple of 64; zero tokens is still a no-op
+    assert f(FAKE, FAKE, FAKE, FAKE, 4, 1, 8, 64, FAKE, 1, None) == bad                      # set
+    assert f(FAKE, FAKE, FAKE, FAKE, 3, 17, 8, 64, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 3, 2, 8, 48, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
+    assert f(None, None, None, None, 3, 0, 8, 64, None, 1, None) == q.QIFT_OK
 
 
 def test_python_binding_refuses_cpu_tensors():

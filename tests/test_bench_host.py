@@ -13,6 +13,8 @@ def test_linear_bytes_q_proj_decode():
     # codes + w scales + int8 activations + act scale + fp16 output for 4096x4096, one token
     assert bench.linear_bytes(1, 4096, 4096, 2) == 4096 * 4096 // 4 + 4 * 4096 + 4096 + 4 + 2 * 4096
     assert bench.acts_bytes(1, 4096) == 3 * 4096 + 4
+    # 4-bit weights: half a byte of codes per weight
+    assert bench.linear_bytes(1, 4096, 4096, 2, "int4") == 4096 * 4096 // 2 + 4 * 4096 + 4096 + 4 + 2 * 4096
 
 
 def test_peaks_reads_measured_file_or_fallback():

@@ -166,6 +166,117 @@ def test_rotate_quantize_weights_block0_and_bad_block():
             qg.qift_rotate_quantize_weights(dev(w), bad, "qift")
 
 
+# ----------------------------------------------------------------- W4A4 (4-bit weights)
+@pytest.mark.parametrize("n_out,n_in,block", [(5, 16, 16), (33, 48, 16), (64, 512, 128), (40, 4096, 4096),
+                                               (9, 11008, 128), (7, 3072, 128)])
+def test_quantize_weights_w4_parity(n_out, n_in, block):
+    w = oracle.rotate_f32(synth.weights(n_out, n_in, (n_in, 13)), block)
+    codes, scales, mse, _ = oracle.quantize_weights_w4(w)
+    gc, gs, gm = qg.qift_quantize_weights(dev(w), "int4")
+    assert gc.shape == (n_out, n_in // 8)
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+    assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+    raw = synth.weights(n_out, n_in, (n_in, 13))
+    fc, fs, fm = qg.qift_rotate_quantize_weights(dev(raw), block, "int4")
+    assert torch.equal(fc, gc) and torch.equal(fs, gs) and torch.equal(fm, gm)
+
+
+def test_quantize_weights_w4_edge_rows():
+    # zero row, one outlier, signed zeros, exact midpoints (j + 0.5) s, a constant row
+    K = 64
+    w = np.zeros((6, K), np.float32)
+    w[1, 7] = 1e3
+    w[1, 8:] = 1e-3
+    w[2, :] = -0.0
+    w[2, 3] = 0.5
+    w[3, :] = np.float32(0.25)
+    w[4, 0] = np.float32(1.75)                                  # s = 0.25 at f = 1
+    w[4, 1:8] = [(j + 0.5) * 0.25 for j in range(7)]
+    w[4, 8:15] = [-(j + 0.5) * 0.25 for j in range(7)]
+    w[5] = synth.weights(1, K, (98,))[0]
+    for grid, lo, hi in ((100, 0.2, 1.0), (2, 1.0, 1.0), (256, 0.05, 4.0)):
+        codes, scales, mse, _ = oracle.quantize_weights_w4(w, grid, lo, hi)
+        gc, gs, gm = qg.qift_quantize_weights(dev(w), "int4", grid, lo, hi)
+        assert np.array_equal(codes_u32(gc), codes), grid
+        assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+        assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
+def _linear_w4_case(T, N, K, seed, out_dtype):
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-7, 8, size=(T, K)).astype(np.int8)
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    s_a = rng.uniform(0.1, 2.0, T).astype(np.float32)
+    npdt = np.float16 if out_dtype == torch.float16 else np.float32
+    y, _ = oracle.linear_w4(q, s_a, codes, s_w, npdt)
+    gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), "int4", out_dtype)
+    return host(gy), y
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8, 9, 16])
+@pytest.mark.parametrize("N,K", [(1, 64), (37, 64), (129, 4096), (4096, 4096), (17, 14336), (300, 11008),
+                                 (9, 32768)])
+def test_linear_w4_parity(T, N, K):
+    for out_dtype in (torch.float32, torch.float16):
+        got, ref = _linear_w4_case(T, N, K, T * 7919 + N + K, out_dtype)
+        tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
+        u = np.uint16 if out_dtype == torch.float16 else np.uint32
+        assert np.array_equal(got.view(u), ref.view(u))
+
+
+def test_linear_w4_extreme_accumulators():
+    # activations +-7 against the outer levels +-7 (codes 14 and 0): |acc| = 49 K at K = 32768
+    T, N, K = 3, 8, 32768
+    q = np.full((T, K), 7, np.int8)
+    q[1] = -7
+    q[2, ::2] = -7
+    codes = np.full((N, K // 8), 0xEEEEEEEE, np.uint32)
+    codes[1::2] = 0
+    s_w = np.ones(N, np.float32)
+    s_a = np.ones(T, np.float32)
+    y, acc = oracle.linear_w4(q, s_a, codes, s_w, np.float32)
+    assert np.abs(acc).max() == 49 * K
+    gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), "int4", torch.float32)
+    assert np.array_equal(host(gy), y)
+
+
+def test_linear_w4_unsupported_shapes_and_decode():
+    rng = np.random.default_rng(1)
+    K, N = 128, 16
+    codes = dev(rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32).view(np.int32))
+    s_w = dev(np.ones(N, np.float32))
+    for T in (17, 64):                                         # more tokens than the 4-bit kernel takes
+        q = dev(np.zeros((T, K), np.int8))
+        with pytest.raises(qg.QiftError):
+            qg.qift_linear(q, dev(np.ones(T, np.float32)), codes, s_w, "int4", torch.float32)
+    q48 = dev(np.zeros((2, 48), np.int8))                      # n_in not a multiple of 64
+    with pytest.raises(qg.QiftError):
+        qg.qift_linear(q48, dev(np.ones(2, np.float32)), dev(np.zeros((N, 6), np.int32)), s_w, "int4")
+    with pytest.raises(qg.QiftError):                          # no one-launch decode for 4-bit weights
+        qg.qift_decode_linear(dev(np.zeros((1, K), np.float16)), 128, codes, s_w, "int4")
+    y = qg.qift_linear(dev(np.zeros((0, K), np.int8)), dev(np.ones(0, np.float32)), codes, s_w, "int4")
+    assert y.shape == (0, N)
+
+
+@pytest.mark.parametrize("T,N,K,block", [(1, 256, 512, 128), (4, 1000, 4096, 128), (16, 64, 16384, 4096),
+                                         (5, 96, 14336, 1024)])
+def test_w4a4_path_end_to_end(T, N, K, block):
+    # raw weights and fp16 tokens through rotation, 4-bit weights, INT4 tokens and the W4A4 linear
+    W = synth.weights(N, K, (N, K, 17))
+    x = synth.activations(T, K, (T, K, 17), n_outliers=synth.outlier_count(K))
+    codes, scales, _, _ = oracle.quantize_weights_w4(oracle.rotate_f32(W, block))
+    q, s_a, _ = oracle.quantize_acts(x, block)
+    ref, _ = oracle.linear_w4(q, s_a, codes, scales, np.float32)
+    gc, gs, _ = qg.qift_rotate_quantize_weights(dev(W), block, "int4")
+    gq, gsa = qg.qift_quantize_acts(dev(x), block)
+    gy = qg.qift_linear(gq, gsa, gc, gs, "int4", torch.float32)
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gq), q)
+    assert np.array_equal(host(gy), ref)
+
+
 # ------------------------------------------------------------------- KV4 (packed INT4 K/V)
 @pytest.mark.parametrize("T,n,block", [(1, 128, 128), (7, 1024, 128), (300, 4096, 128), (16, 4096, 4096),
                                        (5, 64, 0), (33, 8192, 64), (2, 16384, 128), (3, 1024, 1024)])

@@ -31,7 +31,8 @@ def host(t):
 
 
 CASES = [(wl.name, i) for wl in (synth.SINGLE_256x512, synth.LLAMA7B_QPROJ_DECODE, synth.LLAMA7B_MLP_PREFILL,
-                                 synth.LLAMA31_8B_MLP_DECODE16) for i in range(len(wl.linears))]
+                                 synth.LLAMA31_8B_MLP_DECODE16, synth.LLAMA7B_QPROJ_DECODE_W4,
+                                 synth.LLAMA31_8B_MLP_DECODE16_W4) for i in range(len(wl.linears))]
 
 
 @pytest.mark.parametrize("wname,idx", CASES)
@@ -56,9 +57,13 @@ def test_workload_linear_parity(wname, idx):
     rows = np.sort(rng.choice(N, size=min(N, 96), replace=False))
     toks = np.sort(rng.choice(T, size=min(T, 24), replace=False))
     o_wrot = oracle.rotate_f32(W[rows], wl.w_block)
-    o_codes, o_scales, _, _ = oracle.quantize_weights(o_wrot, wl.levelset)
     o_q, o_sa, _ = oracle.quantize_acts(x[toks], wl.a_block)
-    o_y, _ = oracle.linear(o_q, o_sa, o_codes, o_scales, wl.levelset, np_dt)
+    if wl.levelset == "int4":
+        o_codes, o_scales, _, _ = oracle.quantize_weights_w4(o_wrot)
+        o_y, _ = oracle.linear_w4(o_q, o_sa, o_codes, o_scales, np_dt)
+    else:
+        o_codes, o_scales, _, _ = oracle.quantize_weights(o_wrot, wl.levelset)
+        o_y, _ = oracle.linear(o_q, o_sa, o_codes, o_scales, wl.levelset, np_dt)
 
     assert np.array_equal(w_rot[rows].view(np.uint32), o_wrot.view(np.uint32))
     assert np.array_equal(gc[rows], o_codes)

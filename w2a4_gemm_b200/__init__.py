@@ -21,9 +21,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqift.so")
 
 QIFT_OK, QIFT_ERR_INVALID_ARG, QIFT_ERR_UNSUPPORTED, QIFT_ERR_CUDA, QIFT_ERR_TIMEOUT = range(5)
-QIFT_SET_QIFT, QIFT_SET_POT, QIFT_SET_STD = 0, 1, 2
+QIFT_SET_QIFT, QIFT_SET_POT, QIFT_SET_STD, QIFT_SET_INT4 = 0, 1, 2, 3
 QIFT_F32, QIFT_F16 = 0, 1
-LEVELSETS = {"qift": QIFT_SET_QIFT, "pot": QIFT_SET_POT, "std": QIFT_SET_STD}
+LEVELSETS = {"qift": QIFT_SET_QIFT, "pot": QIFT_SET_POT, "std": QIFT_SET_STD, "int4": QIFT_SET_INT4}
 
 _lib = None
 
@@ -102,6 +102,11 @@ def _set(levelset) -> int:
     return LEVELSETS[levelset] if isinstance(levelset, str) else int(levelset)
 
 
+def _codes_per_word(levelset) -> int:
+    """Codes per 32-bit word: 16 two-bit codes, or 8 four-bit codes for the INT4 set."""
+    return 8 if _set(levelset) == QIFT_SET_INT4 else 16
+
+
 def qift_rotate(x: torch.Tensor, block: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Block-diagonal normalised Walsh-Hadamard rotation along the last axis (fp32 or fp16)."""
     _cuda(x, "x")
@@ -117,14 +122,15 @@ def qift_rotate(x: torch.Tensor, block: int, out: torch.Tensor | None = None, st
 
 def qift_quantize_weights(w_rot: torch.Tensor, levelset="qift", grid_points: int = 100, lo: float = 0.2,
                           hi: float = 1.0, with_mse: bool = True, stream=None):
-    """Per-row scale search + nearest-level encode + 2-bit pack.
+    """Per-row scale search + nearest-level encode + 2-bit pack (4-bit for ``"int4"``).
 
-    Returns ``(codes int32-viewed-as-u32 [N, K/16], scales f32 [N], row_mse f64 [N] or None)``.
+    Returns ``(codes int32-viewed-as-u32 [N, K/16] ([N, K/8] for "int4"), scales f32 [N],
+    row_mse f64 [N] or None)``.
     """
     _cuda(w_rot, "w_rot", torch.float32)
     n_out, n_in = w_rot.shape
     dev = w_rot.device
-    codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
+    codes = torch.empty((n_out, n_in // _codes_per_word(levelset)), dtype=torch.int32, device=dev)
     scales = torch.empty(n_out, dtype=torch.float32, device=dev)
     mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
     _check(lib().qift_quantize_weights(_ptr(w_rot), n_out, n_in, _set(levelset), grid_points, lo, hi,
@@ -140,7 +146,7 @@ def qift_rotate_quantize_weights(w: torch.Tensor, block: int, levelset="qift", g
     _cuda(w, "w", torch.float32)
     n_out, n_in = w.shape
     dev = w.device
-    codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
+    codes = torch.empty((n_out, n_in // _codes_per_word(levelset)), dtype=torch.int32, device=dev)
     scales = torch.empty(n_out, dtype=torch.float32, device=dev)
     mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
     _check(lib().qift_rotate_quantize_weights(_ptr(w), n_out, n_in, block, _set(levelset), grid_points, lo, hi,
@@ -186,7 +192,8 @@ def qift_dequantize_kv(packed: torch.Tensor, scales: torch.Tensor, block: int, s
 
 def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w_scale: torch.Tensor,
                 levelset="qift", out_dtype=torch.float16, out: torch.Tensor | None = None, stream=None):
-    """Fused W2A4 linear: ``y[t, n] = ((float)acc * w_scale[n]) * act_scale[t]``."""
+    """Fused W2A4 linear (W4A4 for ``"int4"``, 1..16 tokens):
+    ``y[t, n] = ((float)acc * w_scale[n]) * act_scale[t]``."""
     _cuda(q, "q", torch.int8)
     _cuda(act_scale, "act_scale", torch.float32)
     _cuda(codes, "codes")
@@ -195,8 +202,9 @@ def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w
         raise ValueError("codes must be 32-bit words")
     T, K = q.shape
     N = codes.shape[0]
-    if codes.shape[1] * 16 != K:
-        raise ValueError("codes must be [n_out, n_in/16]")
+    cpw = _codes_per_word(levelset)
+    if codes.shape[1] * cpw != K:
+        raise ValueError(f"codes must be [n_out, n_in/{cpw}]")
     y = torch.empty((T, N), dtype=out_dtype, device=q.device) if out is None else _cuda(out, "out", out_dtype)
     dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
     _check(lib().qift_linear(_ptr(q), _ptr(act_scale), _ptr(codes), _ptr(w_scale), _set(levelset), T, N, K,
@@ -213,8 +221,9 @@ def qift_decode_linear(x: torch.Tensor, block: int, codes: torch.Tensor, w_scale
     _cuda(w_scale, "w_scale", torch.float32)
     T, K = x.shape
     N = codes.shape[0]
-    if codes.shape[1] * 16 != K:
-        raise ValueError("codes must be [n_out, n_in/16]")
+    cpw = _codes_per_word(levelset)
+    if codes.shape[1] * cpw != K:
+        raise ValueError(f"codes must be [n_out, n_in/{cpw}]")
     y = torch.empty((T, N), dtype=out_dtype, device=x.device) if out is None else _cuda(out, "out", out_dtype)
     if q_out is not None:
         _cuda(q_out, "q_out", torch.int8)

@@ -70,7 +70,8 @@ qift_status qift_rotate(const void* x, void* y, qift_dtype dt, int64_t rows, int
 qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_in, qift_levelset set,
                                   int32_t grid_points, double lo, double hi, uint32_t* codes, float* scales,
                                   double* row_mse, void* stream) {
-    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD && set != QIFT_SET_INT4)
+        return QIFT_ERR_INVALID_ARG;
     if (n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
     if (grid_points < 2 || grid_points > 256) return QIFT_ERR_INVALID_ARG;
     if (!(lo > 0.0) || !(hi >= lo) || !(hi <= 4.0)) return QIFT_ERR_INVALID_ARG;
@@ -87,7 +88,8 @@ qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_i
 qift_status qift_rotate_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int32_t block,
                                          qift_levelset set, int32_t grid_points, double lo, double hi,
                                          uint32_t* codes, float* scales, double* row_mse, void* stream) {
-    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD && set != QIFT_SET_INT4)
+        return QIFT_ERR_INVALID_ARG;
     if (n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
     if (block != 0 && (!valid_block(block) || n_in % block != 0)) return QIFT_ERR_INVALID_ARG;
     if (grid_points < 2 || grid_points > 256) return QIFT_ERR_INVALID_ARG;
@@ -142,17 +144,21 @@ qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64
 qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint32_t* codes, const float* w_scale,
                         qift_levelset set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, qift_dtype out_dt,
                         void* stream) {
-    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD && set != QIFT_SET_INT4)
+        return QIFT_ERR_INVALID_ARG;
     if (out_dt != QIFT_F32 && out_dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
     if (tokens < 0 || n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
     if (set == QIFT_SET_STD) return QIFT_ERR_UNSUPPORTED;
     if (n_in > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (set == QIFT_SET_INT4 && !qift::linear_w4_supported(tokens == 0 ? 1 : tokens, n_in)) return QIFT_ERR_UNSUPPORTED;
     if (tokens == 0 || n_out == 0) return QIFT_OK;
     if (!q_act || !act_scale || !codes || !w_scale || !y) return QIFT_ERR_INVALID_ARG;
     if (!aligned16(q_act) || !aligned16(codes) || !aligned16(y) || !aligned4(act_scale) || !aligned4(w_scale))
         return QIFT_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f16 = out_dt == QIFT_F16;
+    if (set == QIFT_SET_INT4)  // one kernel family for 4-bit weights, whatever the debug pin
+        return from_cuda(qift::launch_linear_w4(q_act, act_scale, codes, w_scale, tokens, n_out, n_in, y, f16, s));
     int path = qift::debug_linear_path();
     if (path == qift::kPathAuto) {
         if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
@@ -195,7 +201,9 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
 qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int32_t block, const uint32_t* codes,
                                const float* w_scale, qift_levelset set, int64_t n_out, void* y, qift_dtype out_dt,
                                int8_t* q_out, float* act_scale_out, void* stream) {
-    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD) return QIFT_ERR_INVALID_ARG;
+    if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD && set != QIFT_SET_INT4)
+        return QIFT_ERR_INVALID_ARG;
+    if (set == QIFT_SET_INT4) return QIFT_ERR_UNSUPPORTED;
     if (out_dt != QIFT_F32 && out_dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
     if (tokens < 0 || n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
     if (block != 0 && (!valid_block(block) || n_in % block != 0)) return QIFT_ERR_INVALID_ARG;

@@ -89,6 +89,11 @@ void debug_set_one_token_wait_limit(long long cycles);
 void debug_stall_next_one_token();
 cudaError_t read_and_clear_one_token_error(int* word);
 
+// 4-bit weights (QIFT_SET_INT4), 1..16 tokens: CUDA-core W4A4 GEMV.
+bool linear_w4_supported(int64_t tokens, int64_t n_in);
+cudaError_t launch_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                             int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16, cudaStream_t s);
+
 // Test hooks behind qift_debug.h.
 enum LinearPath {
     kPathAuto = 0,

@@ -27,8 +27,12 @@ namespace qift {
 template <int SET>
 struct Encoder {
     float s, thr1, thr2, l_in, l_out;
+    float thr[7];  // W4: midpoints (j + 0.5) s rounded down, j = 0..6
     __device__ __forceinline__ explicit Encoder(float s_) : s(s_) {
-        if constexpr (SET == kSetQift) {        // levels +-0.5 s, +-1.5 s; midpoint s
+        if constexpr (SET == kSetInt4) {        // levels {-7..7} s; midpoints (j + 0.5) s
+#pragma unroll
+            for (int j = 0; j < 7; ++j) thr[j] = __fmul_rd((float)j + 0.5f, s);
+        } else if constexpr (SET == kSetQift) {  // levels +-0.5 s, +-1.5 s; midpoint s
             thr1 = s;
             l_in = __fmul_rn(0.5f, s);
             l_out = __fmul_rn(1.5f, s);
@@ -41,9 +45,20 @@ struct Encoder {
             thr2 = __fmul_rd(0.5f, s);
         }
     }
-    // Code 0..3 (monotone in level).  Ties go to the smaller magnitude; w >= 0 is positive.
+    // W4: the level's magnitude -- the number of midpoints strictly below |w| (ties stay low).
+    __device__ __forceinline__ int w4_mag(float a) const {
+        int j = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) j += a > thr[i] ? 1 : 0;
+        return j;
+    }
+    // Code (monotone in level): 0..3, or u = level + 7 in 0..14 for W4.  Ties go to the smaller
+    // magnitude; w >= 0 is positive.
     __device__ __forceinline__ uint32_t code(float w) const {
-        if constexpr (SET == kSetStd) {
+        if constexpr (SET == kSetInt4) {
+            const int j = w4_mag(fabsf(w));
+            return (uint32_t)(w >= 0.0f ? 7 + j : 7 - j);
+        } else if constexpr (SET == kSetStd) {
             const float nw = -w;
             if (nw > thr1) return 0u;   // w < -1.5 s
             if (nw > thr2) return 1u;   // w < -0.5 s
@@ -57,7 +72,12 @@ struct Encoder {
     // Squared reconstruction error of w, in fp32, for its code.
     __device__ __forceinline__ float sq_err(float w) const {
         float e;
-        if constexpr (SET == kSetStd) {
+        if constexpr (SET == kSetInt4) {
+            const float a = fabsf(w);
+            // (float)j by the exact magic-number add (j <= 7), off the conversion unit
+            const float jf = __fsub_rn(__int_as_float(0x4B400000 + w4_mag(a)), 12582912.0f);
+            e = __fsub_rn(a, __fmul_rn(jf, s));
+        } else if constexpr (SET == kSetStd) {
             const float l = __fmul_rn((float)((int)code(w) - 2), s);
             e = __fsub_rn(w, l);
         } else {
@@ -199,7 +219,7 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
     __syncthreads();
 
     // Candidate scales, binary64 in the order lo + ((hi - lo) * k) / (G - 1), then * m / L.
-    const double lambda = SET == kSetQift ? 1.5 : (SET == kSetPot ? 4.0 : 2.0);
+    const double lambda = SET == kSetQift ? 1.5 : (SET == kSetPot ? 4.0 : (SET == kSetInt4 ? 7.0 : 2.0));
     for (int f = tid; f < rows * G; f += nthr) {
         const int r = f / G, g = f - r * G;
         const double fr = __dadd_rn(lo, __ddiv_rn(__dmul_rn(__dsub_rn(hi, lo), (double)g), (double)(G - 1)));
@@ -235,22 +255,24 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
     }
     __syncthreads();
 
-    // Encode and pack: word j holds the codes of inputs 16j .. 16j+15, 2 bits each.
+    // Encode and pack: word j holds the codes of inputs CPW*j .. CPW*j + CPW-1, least
+    // significant first -- 16 codes of 2 bits, or (W4) 8 codes of 4 bits.
+    constexpr int CPW = SET == kSetInt4 ? 8 : 16, BITS = 32 / CPW;
     for (int r = 0; r < rows; ++r) {
         const int b = best_s[r];
         const float sr = cand[r * kQwMaxG + b];
         const Encoder<SET> enc(sr);
-        uint32_t* crow = codes + (row0 + r) * (K / 16);
-        for (int64_t j = tid; j < K / 16; j += nthr) {
-            const float4* w4 = reinterpret_cast<const float4*>(ws + r * K + j * 16);
+        uint32_t* crow = codes + (row0 + r) * (K / CPW);
+        for (int64_t j = tid; j < K / CPW; j += nthr) {
+            const float4* w4 = reinterpret_cast<const float4*>(ws + r * K + j * CPW);
             uint32_t word = 0;
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
+            for (int v4 = 0; v4 < CPW / 4; ++v4) {
                 const float4 v = w4[v4];
-                word |= enc.code(v.x) << (8 * v4);
-                word |= enc.code(v.y) << (8 * v4 + 2);
-                word |= enc.code(v.z) << (8 * v4 + 4);
-                word |= enc.code(v.w) << (8 * v4 + 6);
+                word |= enc.code(v.x) << (BITS * (4 * v4));
+                word |= enc.code(v.y) << (BITS * (4 * v4 + 1));
+                word |= enc.code(v.z) << (BITS * (4 * v4 + 2));
+                word |= enc.code(v.w) << (BITS * (4 * v4 + 3));
             }
             crow[j] = word;
         }
@@ -293,6 +315,7 @@ cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in,
         case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
         case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
         case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
+        case kSetInt4: return launch_qw<kSetInt4>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
         default: return cudaErrorInvalidValue;
     }
 }

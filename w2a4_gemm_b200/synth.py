@@ -62,7 +62,7 @@ class Linear:
 class Workload:
     name: str
     description: str
-    levelset: str                 # "qift" | "pot" | "std"
+    levelset: str                 # "qift" | "pot" | "std" | "int4" (4-bit weights, W4A4)
     w_block: int                  # Hadamard block on the weights' input dimension
     a_block: int                  # Hadamard block on the activations (same as w_block)
     tokens: int
@@ -118,8 +118,28 @@ LLAMA31_8B_MLP_DECODE16 = Workload(
              Linear("down_proj", 4096, 14336, (4, 2), (104, 2))),
 )
 
+# The 4-bit layers of the mixed W2/W4 configuration, at the same decode shapes.
+LLAMA7B_QPROJ_DECODE_W4 = Workload(
+    name="llama7b_q_proj_decode_T1_w4",
+    description="LLaMA-7B q_proj decode GEMV 4096x4096, 1 token, full 4096-point Hadamard, 4-bit weights (W4A4)",
+    levelset="int4", w_block=4096, a_block=4096, tokens=1, out_dtype="f16", w_dist="t4",
+    n_outliers=-1,
+    linears=(Linear("q_proj", 4096, 4096, (2,), (102,)),),
+)
+
+LLAMA31_8B_MLP_DECODE16_W4 = Workload(
+    name="llama31_8b_mlp_decode_T16_w4",
+    description="LLaMA-3.1-8B MLP decode at 16 tokens: up/gate 14336x4096, down 4096x14336, "
+                "128-block Hadamard, 4-bit weights (W4A4)",
+    levelset="int4", w_block=128, a_block=128, tokens=16, out_dtype="f16", w_dist="t4",
+    n_outliers=0,
+    linears=(Linear("gate_proj", 14336, 4096, (4, 0), (104, 0)),
+             Linear("up_proj", 14336, 4096, (4, 1), (104, 0)),
+             Linear("down_proj", 4096, 14336, (4, 2), (104, 2))),
+)
+
 WORKLOADS = {w.name: w for w in (SINGLE_256x512, LLAMA7B_QPROJ_DECODE, LLAMA7B_MLP_PREFILL,
-                                 LLAMA31_8B_MLP_DECODE16)}
+                                 LLAMA31_8B_MLP_DECODE16, LLAMA7B_QPROJ_DECODE_W4, LLAMA31_8B_MLP_DECODE16_W4)}
 
 # Offline quantization of a full 8B-shaped model: 32 layers x 7 linear modules.
 MODEL_8B_PROJS = (("q_proj", 4096, 4096), ("k_proj", 1024, 4096), ("v_proj", 1024, 4096),
