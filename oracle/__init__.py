@@ -151,7 +151,8 @@ def quantize_weights_w4(w_rot: np.ndarray, grid_points: int = 100, lo: float = 0
     """W4 per-channel scale search + nearest-level encode + pack (levels {-7..7} * s).
 
     Returns ``(codes uint32 [N, K/8], scales f32 [N], row_mse f64 [N], best_k int32 [N])``;
-    the code of input k is ``level + 7`` at bits ``4*(k%8)`` of word ``k/8``.
+    the code of input k is the level's two's-complement nibble, at bits
+    ``8*(k%4) + 4*((k%8)//4)`` of word ``k/8`` (byte j: input j low, input j+4 high).
     """
     w = np.ascontiguousarray(w_rot, dtype=np.float32)
     n_out, n_in = w.shape
@@ -164,12 +165,22 @@ def quantize_weights_w4(w_rot: np.ndarray, grid_points: int = 100, lo: float = 0
     return codes, scales, mse, best
 
 
+W4_SHIFTS = np.array([8 * (p % 4) + 4 * (p // 4) for p in range(8)], dtype=np.uint32)
+
+
+def pack_w4(levels: np.ndarray) -> np.ndarray:
+    """int levels [N, K] in [-8, 7] -> uint32 [N, K/8] in the W4 word layout."""
+    lv = np.ascontiguousarray(levels).astype(np.int64)
+    nib = (lv & 0xF).astype(np.uint32).reshape(lv.shape[0], -1, 8)
+    return np.bitwise_or.reduce(nib << W4_SHIFTS[None, None, :], axis=2).astype(np.uint32)
+
+
 def unpack_w4(codes: np.ndarray, n_in: int) -> np.ndarray:
-    """uint32 [N, K/8] -> int8 levels [N, K] in [-7, 7]."""
+    """uint32 [N, K/8] -> int8 levels [N, K] (two's-complement nibbles, -8..7)."""
     c = np.ascontiguousarray(codes, dtype=np.uint32)
-    shifts = (4 * np.arange(8, dtype=np.uint32))[None, None, :]
-    u = (c[:, :, None] >> shifts) & np.uint32(0xF)
-    return (u.reshape(c.shape[0], n_in).astype(np.int16) - 7).astype(np.int8)
+    u = (c[:, :, None] >> W4_SHIFTS[None, None, :]) & np.uint32(0xF)
+    u = u.reshape(c.shape[0], n_in).astype(np.int16)
+    return np.where(u >= 8, u - 16, u).astype(np.int8)
 
 
 def linear_w4(q: np.ndarray, s_a: np.ndarray, codes: np.ndarray, s_w: np.ndarray, out_dtype=np.float32):

@@ -263,9 +263,17 @@ int qo_unpack_codes(const uint32_t* codes, int64_t n_out, int64_t n_in, uint8_t*
  *           takes the positive side (R7);
  *   error:  e = |w| - l, l = j * s in binary32, e * e in binary32, summed in binary64 in index
  *           order (R9);
- *   code:   u = level + 7 in [0, 14], eight per u32, the code of input k at bits 4*(k%8) .. +3,
- *           least significant first (R21).  The stored scale is s itself.
+ *   code:   the level as a 4-bit two's-complement nibble, eight per u32 (R21): word k/8 holds
+ *           inputs 8w .. 8w+7, byte j of it input 8w+j in the low nibble and input 8w+j+4 in
+ *           the high nibble, i.e. input k at bits 8*(k%4) + 4*((k%8)/4) .. +3.  The stored
+ *           scale is s itself.
  * ------------------------------------------------------------------------------------- */
+/* Bit position of input k's nibble inside its word (R21). */
+static int w4_shift(int64_t k) { return (int)(8 * (k % 4) + 4 * ((k % 8) / 4)); }
+
+/* The level a nibble stores: its two's-complement value, -8..7. */
+static int32_t w4_level(uint32_t nibble) { return nibble >= 8u ? (int32_t)nibble - 16 : (int32_t)nibble; }
+
 static int32_t encode_w4(float w, float s) {
     const double a = fabs((double)w), sd = (double)s;
     int32_t j = 0;
@@ -319,7 +327,7 @@ int qo_quantize_weights_w4(const float* w, int64_t n_out, int64_t n_in, int32_t 
         uint32_t* out = codes + n * words;
         for (int64_t j = 0; j < words; ++j) out[j] = 0u;
         for (int64_t k = 0; k < n_in; ++k)
-            out[k / 8] |= (uint32_t)(encode_w4(row[k], s) + 7) << (4 * (k % 8));
+            out[k / 8] |= ((uint32_t)encode_w4(row[k], s) & 0xFu) << w4_shift(k);
         scales[n] = s;
         if (row_mse) row_mse[n] = best / (double)n_in;
         if (best_k) best_k[n] = kbest;
@@ -327,7 +335,7 @@ int qo_quantize_weights_w4(const float* w, int64_t n_out, int64_t n_in, int32_t 
     return bad ? -2 : 0;
 }
 
-/* W4A4 linear: acc[t][n] = sum_k q[t][k] * (u(code) - 7) exactly (int64, must fit int32), then
+/* W4A4 linear: acc[t][n] = sum_k q[t][k] * level(code) exactly (int64, must fit int32), then
  * y = ((float)acc * s_w[n]) * s_a[t] (R13).  acc and y may be NULL. */
 int qo_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int64_t tokens,
                  int64_t n_out, int64_t n_in, int32_t* acc_out, float* y) {
@@ -339,8 +347,8 @@ int qo_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const
         for (int64_t n = 0; n < n_out; ++n) {
             int64_t sum = 0;
             for (int64_t k = 0; k < n_in; ++k) {
-                const int32_t u = (int32_t)((codes[n * words + k / 8] >> (4 * (k % 8))) & 0xFu);
-                sum += (int64_t)q[t * n_in + k] * (int64_t)(u - 7);
+                const uint32_t nib = (codes[n * words + k / 8] >> w4_shift(k)) & 0xFu;
+                sum += (int64_t)q[t * n_in + k] * (int64_t)w4_level(nib);
             }
             if (sum > INT32_MAX || sum < INT32_MIN) {
 #pragma omp atomic write

@@ -59,14 +59,37 @@ def test_midpoint_ties_and_signed_zero():
 
 
 def test_packing_hand_word():
-    # levels -7, 0, 7, 1, -1, 3, -3, 6 -> codes u = level + 7 = 0, 7, 14, 8, 6, 10, 4, 13, four
-    # bits each from the least significant end: 0xD4A68E70.
+    # levels -7, 0, 7, 1 (inputs 0..3) and -1, 3, -3, 6 (inputs 4..7) as two's-complement
+    # nibbles 9, 0, 7, 1 and F, 3, D, 6; byte j = input j | input j+4 << 4:
+    #   0xF9, 0x30, 0xD7, 0x61 -> 0x61D730F9.
     levels = np.array([-7, 0, 7, 1, -1, 3, -3, 6], dtype=np.float32)
     w = np.concatenate([levels * np.float32(0.25)] * 2)[None, :]    # max |w| = 1.75 -> s = 0.25
     codes, scales, _, _ = oracle.quantize_weights_w4(w, grid_points=2, lo=1.0, hi=1.0)
     assert scales[0] == np.float32(0.25)
-    assert codes.tolist() == [[0xD4A68E70, 0xD4A68E70]]
+    assert codes.tolist() == [[0x61D730F9, 0x61D730F9]]
     assert oracle.unpack_w4(codes, 16).tolist() == [levels.astype(int).tolist() * 2]
+    assert oracle.pack_w4(levels.astype(int)[None, :]).tolist() == [[0x61D730F9]]
+
+
+def _pack_by_hand(lv: np.ndarray) -> np.ndarray:
+    """Bit by bit: input k of a row goes to word k // 8, byte k % 4, high nibble when k % 8 >= 4."""
+    N, K = lv.shape
+    out = np.zeros((N, K // 8), np.uint32)
+    for n in range(N):
+        for k in range(K):
+            nib = int(lv[n, k]) % 16
+            out[n, k // 8] |= np.uint32(nib << (8 * (k % 4) + (4 if k % 8 >= 4 else 0)))
+    return out
+
+
+def test_nibble_sign_and_byte_scaling():
+    # Every nibble reads as its two's-complement level, and the nibble moved to the top of a
+    # byte reads, as a signed byte, 16 times that level (the form a signed dp4a consumes).
+    for nib in range(16):
+        level = nib - 16 if nib >= 8 else nib
+        word = np.array([[nib << 4 | nib]], np.uint32)            # inputs 0 (low) and 4 (high)
+        assert oracle.unpack_w4(np.array([[word[0, 0]]], np.uint32), 8)[0, [0, 4]].tolist() == [level, level]
+        assert int(np.uint8(nib << 4).view(np.int8)) == 16 * level
 
 
 def test_scale_search_is_grid_optimal():
@@ -88,18 +111,14 @@ def test_scale_search_is_grid_optimal():
 def test_linear_w4_is_integer_matmul(T, N, K):
     rng = np.random.default_rng(T + N + K)
     q = rng.integers(-7, 8, size=(T, K)).astype(np.int8)
-    u = rng.integers(0, 15, size=(N, K)).astype(np.uint32)
-    codes = np.zeros((N, K // 8), np.uint32)
-    for k in range(K):
-        codes[:, k // 8] |= u[:, k] << np.uint32(4 * (k % 8))
+    lv = rng.integers(-8, 8, size=(N, K)).astype(np.int64)       # every nibble, -8 included
+    codes = _pack_by_hand(lv)
+    assert np.array_equal(oracle.pack_w4(lv), codes)
     s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
     s_a = rng.uniform(0.1, 2.0, T).astype(np.float32)
     y, acc = oracle.linear_w4(q, s_a, codes, s_w)
-    lv = u.astype(np.int64) - 7
     ref = q.astype(np.int64) @ lv.T
     assert np.array_equal(acc.astype(np.int64), ref)
-    # the offset identity the GPU path uses: sum q (u - 7) = sum q u - 7 sum q
-    assert np.array_equal(ref, q.astype(np.int64) @ u.astype(np.int64).T - 7 * q.astype(np.int64).sum(1, keepdims=True))
     yr = ((acc.astype(np.float32) * s_w[None, :]).astype(np.float32) * s_a[:, None]).astype(np.float32)
     assert np.array_equal(y, yr)
 
