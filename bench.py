@@ -62,15 +62,17 @@ def peaks():
 # as null.  `scale` converts the captured launch to the benchmarked one when the shapes differ
 # (traffic grows in proportion to the weights processed).
 PROFILED_TRAFFIC = {
-    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="b6667d172c58909a", bytes=4231168 + 0,
+    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="7072e2cc258b4f58", bytes=4231168 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
-    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="1cb8a9e37443764c",
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="0401423015962d76",
                     bytes=19752192 + 1284864, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
-    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="312551652af22a8e", bytes=14854144 + 0,
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="efcfee8669e604e6", bytes=14854144 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
-    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="cb68d6cdb915937a",
-                    bytes=67147008 + 1017088, scale=14336 * 4096 / (4096 * 4096),
+    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="7caa8a2d0ba3cce3",
+                    bytes=67147776 + 1114368, scale=14336 * 4096 / (4096 * 4096),
                     profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
+    "decode16_w4": dict(files=("linear_w4.cu", "common.cuh"), sha="19e2960b712910c4", bytes=29504000 + 0,
+                        profile="profiles/w4_gemv_kernel_mlp_decode_T16_w4.md"),
 }
 
 

@@ -41,7 +41,7 @@ typedef enum {
 
 /* Level sets.  The 2-bit codes 0..3 map to levels in increasing order (code 0 = most
  * negative).  QIFT_SET_INT4 is the 4-bit set of the Abstract's mixed W2/W4 layers: levels
- * {-7, ..., +7} * s stored as u = level + 7 (0..14), eight codes per 32-bit word. */
+ * {-7, ..., +7} * s stored as two's-complement nibbles, eight per 32-bit word. */
 typedef enum {
     QIFT_SET_QIFT = 0, /* {-3, -1, +1, +3} * t, t = s/2  (= {-1.5, -0.5, +0.5, +1.5} * s) */
     QIFT_SET_POT = 1,  /* {-4, -1, +1, +4} * t  (power of two: sign and shift)             */
@@ -75,9 +75,10 @@ qift_status qift_rotate(const void* x, void* y, qift_dtype dt, int64_t rows, int
  *                in binary64, L = 1.5 (Qift, s-form levels +-0.5 s, +-1.5 s), 4 (PoT), 2 (std).
  *                The usual search is G = 100, lo = 0.2, hi = 1.0.
  *   codes      : u32 [n_out][n_in/16] out.  Code of input k sits in word k/16 at bits
- *                2*(k%16) and 2*(k%16)+1.  QIFT_SET_INT4: u32 [n_out][n_in/8], code of input
- *                k (u = level + 7) in word k/8 at bits 4*(k%8) .. 4*(k%8)+3; L = 7; the nearest
- *                level compares |w| with the midpoints (j + 0.5) s.
+ *                2*(k%16) and 2*(k%16)+1.  QIFT_SET_INT4: u32 [n_out][n_in/8]; the level of
+ *                input k, as a two's-complement nibble, in word k/8 at bits
+ *                8*(k%4) + 4*((k%8)/4) .. +3 (byte j: input j low, input j+4 high); L = 7; the
+ *                nearest level compares |w| with the midpoints (j + 0.5) s.
  *   scales     : fp32 [n_out] out: t = s_best/2 for Qift, s_best for PoT and std, so the
  *                weight is level(code) * t with the integer levels of the set.
  *   row_mse    : fp64 [n_out] out, or NULL: the best candidate's mean squared error.
@@ -145,7 +146,7 @@ qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64
  *   codes     : u32 [n_out][n_in/16], w_scale: fp32 [n_out], from qift_quantize_weights.
  *   set       : QIFT_SET_QIFT or QIFT_SET_POT (QIFT_SET_STD -> QIFT_ERR_UNSUPPORTED), or
  *               QIFT_SET_INT4 (W4A4: codes u32 [n_out][n_in/8]; 1..16 tokens and n_in % 64 == 0,
- *               else QIFT_ERR_UNSUPPORTED; acc = sum q * (u - 7), on CUDA cores).
+ *               else QIFT_ERR_UNSUPPORTED; acc = sum q * level, on CUDA cores).
  *   y         : [tokens][n_out] out, out_dt QIFT_F32 or QIFT_F16 (round to nearest even).
  *   n_in      : multiple of 16, at most 32768 (so |acc| <= 7*4*n_in < 2^24 and (float)acc is
  *               exact).  tokens == 0 or n_out == 0 is a no-op.

@@ -227,13 +227,14 @@ def test_linear_w4_parity(T, N, K):
 
 
 def test_linear_w4_extreme_accumulators():
-    # activations +-7 against the outer levels +-7 (codes 14 and 0): |acc| = 49 K at K = 32768
+    # activations +-7 against the outer levels +7 (nibble 7) and -7 (nibble 9): |acc| = 49 K at
+    # K = 32768
     T, N, K = 3, 8, 32768
     q = np.full((T, K), 7, np.int8)
     q[1] = -7
     q[2, ::2] = -7
-    codes = np.full((N, K // 8), 0xEEEEEEEE, np.uint32)
-    codes[1::2] = 0
+    codes = np.full((N, K // 8), 0x77777777, np.uint32)
+    codes[1::2] = 0x99999999
     s_w = np.ones(N, np.float32)
     s_a = np.ones(T, np.float32)
     y, acc = oracle.linear_w4(q, s_a, codes, s_w, np.float32)

@@ -14,7 +14,7 @@ namespace qift {
 constexpr int kSetQift = 0;
 constexpr int kSetPot = 1;
 constexpr int kSetStd = 2;
-constexpr int kSetInt4 = 3;  // 4-bit weights {-7..7} * s, code u = level + 7, eight per word
+constexpr int kSetInt4 = 3;  // 4-bit weights {-7..7} * s as two's-complement nibbles, eight per word
 
 // Integer level table of a set packed as four signed bytes, byte c = level of code c, so that
 // one byte permute (prmt) turns four 2-bit codes into four int8 weights.

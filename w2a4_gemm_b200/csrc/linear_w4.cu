@@ -1,18 +1,19 @@
-// linear_w4.cu -- qift_linear for 4-bit weights (levels {-7..7} * s, code u = level + 7, eight
-// codes per word) at decode batch sizes (1..16 tokens): a CUDA-core W4A4 GEMV.
+// linear_w4.cu -- qift_linear for 4-bit weights (levels {-7..7} * s per output channel, stored
+// as two's-complement nibbles, eight per word) at decode batch sizes (1..16 tokens): a CUDA-core
+// W4A4 GEMV.
 //
 // "Qift: Shift-Friendly No-Zero W2 Post-Training Quantization for Rotated W2A4/KV4 LLM
 // Inference", Abstract: the evaluation mixes 2-bit and 4-bit layers ("L-layer mixed W2/W4"),
 // both applied to the rotated 4-bit activations.
 //
-//   acc[t][n] = sum_k q[t][k] (u[n][k] - 7) = sum_k q u - 7 sum_k q      (exact, int32)
+//   acc[t][n] = sum_k q[t][k] level[n][k]                                 (exact, int32)
 //   y[t][n]   = ((float)acc * s_w[n]) * s_a[t].
 //
-// The codes are applied without a decode: a word holds inputs 8w..8w+7, nibble i = input i;
-// masking with 0x0F0F0F0F leaves the even inputs' codes in bytes 0..3 and the same mask after a
-// 4-bit shift the odd ones, each meeting the matching activation bytes (gathered with one byte
-// permute) in an unsigned x signed dp4a.  Each lane subtracts 7 * (sum of its activations) from
-// its partial sum before the warp reduction, so the int32 total is exact.
+// The codes are applied without a decode.  Byte j of a word holds input j in its low nibble and
+// input j + 4 in its high nibble, so the word masked with 0xF0F0F0F0 holds, as signed bytes,
+// 16 x the levels of inputs 4..7 and the word shifted left by 4 and masked 16 x those of inputs
+// 0..3: each meets one 32-bit word of INT4 activations in a signed dp4a.  The total is 16 x acc
+// exactly (|16 acc| <= 16 * 8 * 7 * 32768 < 2^31), and an arithmetic shift by 4 recovers acc.
 //
 // Each warp owns R rows and TC tokens; lane l streams 16-byte groups (32 codes) g = l, l+32, ...
 // of its rows.  The codes of the first group are requested before the wait for the previous
@@ -32,12 +33,6 @@ __device__ __forceinline__ void store_out<float>(float* p, float v) { *p = v; }
 template <>
 __device__ __forceinline__ void store_out<__half>(__half* p, float v) { *p = __float2half_rn(v); }
 
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
 template <int R, int TC, typename OutT>
 __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __restrict__ q,
                                                               const float* __restrict__ s_a,
@@ -48,13 +43,11 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
     const int64_t row0 = ((int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5)) * R;
     const int64_t t0 = (int64_t)blockIdx.y * TC;
     const int64_t KW = K / 8, KG = K / 32;  // words and 16-byte groups per row
-    int acc[R][TC], qs[TC];
+    int acc[R][TC];
 #pragma unroll
-    for (int t = 0; t < TC; ++t) {
-        qs[t] = 0;
+    for (int t = 0; t < TC; ++t)
 #pragma unroll
         for (int r = 0; r < R; ++r) acc[r][t] = 0;
-    }
     uint4 cw[R];
     auto load_codes = [&](int64_t g) {
 #pragma unroll
@@ -67,6 +60,17 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
     griddep_wait();
     for (int64_t g = lane; g < KG; g += 32) {
         if (g != lane) load_codes(g);
+        // 16 x levels as signed bytes: lo[r][w] for inputs 8w..8w+3, hi[r][w] for 8w+4..8w+7
+        uint32_t lo[R][4], hi[R][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const uint32_t wd[4] = {cw[r].x, cw[r].y, cw[r].z, cw[r].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                lo[r][w] = (wd[w] << 4) & 0xF0F0F0F0u;
+                hi[r][w] = wd[w] & 0xF0F0F0F0u;
+            }
+        }
 #pragma unroll
         for (int t = 0; t < TC; ++t) {
             uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
@@ -77,25 +81,19 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
             }
             const uint32_t av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {  // word w of the group: inputs 8w .. 8w+7
-                const uint32_t lo = av[2 * w], hi = av[2 * w + 1];
-                const uint32_t ev = prmt(lo, hi, 0x6420u), od = prmt(lo, hi, 0x7531u);
-                qs[t] = dp4a(lo, 0x01010101u, qs[t]);
-                qs[t] = dp4a(hi, 0x01010101u, qs[t]);
+            for (int w = 0; w < 4; ++w)
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    const uint32_t word = w == 0 ? cw[r].x : w == 1 ? cw[r].y : w == 2 ? cw[r].z : cw[r].w;
-                    acc[r][t] = dp4a_us(word & 0x0F0F0F0Fu, ev, acc[r][t]);
-                    acc[r][t] = dp4a_us((word >> 4) & 0x0F0F0F0Fu, od, acc[r][t]);
+                    acc[r][t] = dp4a(lo[r][w], av[2 * w], acc[r][t]);
+                    acc[r][t] = dp4a(hi[r][w], av[2 * w + 1], acc[r][t]);
                 }
-            }
         }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
 #pragma unroll
         for (int t = 0; t < TC; ++t) {
-            const int sum = __reduce_add_sync(0xffffffffu, acc[r][t] - 7 * qs[t]);
+            const int sum = __reduce_add_sync(0xffffffffu, acc[r][t]) >> 4;  // exact: a multiple of 16
             const int64_t n = row0 + r, tt = t0 + t;
             if (lane == ((r * TC + t) & 31) && n < N && tt < T)
                 store_out<OutT>(y + tt * N + n, __fmul_rn(__fmul_rn((float)sum, __ldg(s_w + n)), __ldg(s_a + tt)));
@@ -126,7 +124,7 @@ static cudaError_t dispatch(const int8_t* q, const float* s_a, const uint32_t* c
                             int64_t N, int64_t K, OutT* y, cudaStream_t s) {
     if (T == 1) return launch<2, 1, OutT>(q, s_a, codes, s_w, T, N, K, y, s);
     if (T <= 4) return launch<2, 4, OutT>(q, s_a, codes, s_w, T, N, K, y, s);
-    return launch<1, 8, OutT>(q, s_a, codes, s_w, T, N, K, y, s);
+    return launch<4, 8, OutT>(q, s_a, codes, s_w, T, N, K, y, s);
 }
 
 }  // namespace w4

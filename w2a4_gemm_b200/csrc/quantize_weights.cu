@@ -52,12 +52,12 @@ struct Encoder {
         for (int i = 0; i < 7; ++i) j += a > thr[i] ? 1 : 0;
         return j;
     }
-    // Code (monotone in level): 0..3, or u = level + 7 in 0..14 for W4.  Ties go to the smaller
-    // magnitude; w >= 0 is positive.
+    // Code: 0..3 in increasing level order, or (W4) the level's two's-complement nibble.  Ties go
+    // to the smaller magnitude; w >= 0 is positive.
     __device__ __forceinline__ uint32_t code(float w) const {
         if constexpr (SET == kSetInt4) {
             const int j = w4_mag(fabsf(w));
-            return (uint32_t)(w >= 0.0f ? 7 + j : 7 - j);
+            return (uint32_t)(w >= 0.0f ? j : -j) & 0xFu;
         } else if constexpr (SET == kSetStd) {
             const float nw = -w;
             if (nw > thr1) return 0u;   // w < -1.5 s
@@ -255,9 +255,11 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
     }
     __syncthreads();
 
-    // Encode and pack: word j holds the codes of inputs CPW*j .. CPW*j + CPW-1, least
-    // significant first -- 16 codes of 2 bits, or (W4) 8 codes of 4 bits.
-    constexpr int CPW = SET == kSetInt4 ? 8 : 16, BITS = 32 / CPW;
+    // Encode and pack: word j holds the codes of inputs CPW*j .. CPW*j + CPW-1 -- 16 codes of 2
+    // bits, least significant first, or (W4) 8 nibbles with byte i holding inputs i (low) and
+    // i + 4 (high), so input p of the word sits at bit 8 (p % 4) + 4 (p / 4).
+    constexpr int CPW = SET == kSetInt4 ? 8 : 16;
+    auto shift = [](int p) { return SET == kSetInt4 ? 8 * (p & 3) + 4 * (p >> 2) : 2 * p; };
     for (int r = 0; r < rows; ++r) {
         const int b = best_s[r];
         const float sr = cand[r * kQwMaxG + b];
@@ -269,10 +271,10 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
 #pragma unroll
             for (int v4 = 0; v4 < CPW / 4; ++v4) {
                 const float4 v = w4[v4];
-                word |= enc.code(v.x) << (BITS * (4 * v4));
-                word |= enc.code(v.y) << (BITS * (4 * v4 + 1));
-                word |= enc.code(v.z) << (BITS * (4 * v4 + 2));
-                word |= enc.code(v.w) << (BITS * (4 * v4 + 3));
+                word |= enc.code(v.x) << shift(4 * v4);
+                word |= enc.code(v.y) << shift(4 * v4 + 1);
+                word |= enc.code(v.z) << shift(4 * v4 + 2);
+                word |= enc.code(v.w) << shift(4 * v4 + 3);
             }
             crow[j] = word;
         }
