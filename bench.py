@@ -71,8 +71,6 @@ PROFILED_TRAFFIC = {
     "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="7caa8a2d0ba3cce3",
                     bytes=67147776 + 1114368, scale=14336 * 4096 / (4096 * 4096),
                     profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
-    "decode16_w4": dict(files=("linear_w4.cu", "common.cuh"), sha="19e2960b712910c4", bytes=29504000 + 0,
-                        profile="profiles/w4_gemv_kernel_mlp_decode_T16_w4.md"),
 }
 
 
@@ -348,7 +346,8 @@ def run_ours(args, rank, world):
         unit = "GB/s"
         roof = {"bound": "hbm", "achieved": lin_b / t_lin / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": lin_b / t_lin / 1e9 / pk["hbm_gbs"], "traffic": profiled_traffic(args.workload),
-                "kernel": "qift_linear (W4A4 GEMV)" if wl.levelset == "int4" else "qift_linear (GEMV)",
+                "kernel": ("qift_linear, 4-bit weights (" + ("CUDA-core GEMV" if T == 1 else "tensor-core skinny GEMM")
+                           + ")") if wl.levelset == "int4" else "qift_linear (GEMV)",
                 "peak_source": pk["source"] + " copy bandwidth, burst"}
     else:
         value = world * step_ops * args.steps / secs / 1e12

@@ -215,15 +215,21 @@ def _linear_w4_case(T, N, K, seed, out_dtype):
     return host(gy), y
 
 
+@pytest.mark.parametrize("pin", ["auto", "skinny", "gemv"])   # auto: tensor cores from 2 tokens
 @pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8, 9, 16])
 @pytest.mark.parametrize("N,K", [(1, 64), (37, 64), (129, 4096), (4096, 4096), (17, 14336), (300, 11008),
-                                 (9, 32768)])
-def test_linear_w4_parity(T, N, K):
-    for out_dtype in (torch.float32, torch.float16):
-        got, ref = _linear_w4_case(T, N, K, T * 7919 + N + K, out_dtype)
-        tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
-        u = np.uint16 if out_dtype == torch.float16 else np.uint32
-        assert np.array_equal(got.view(u), ref.view(u))
+                                 (9, 32768), (130, 192)])
+def test_linear_w4_parity(pin, T, N, K):
+    qg.qift_debug_set_linear_path(pin)
+    try:
+        for out_dtype in (torch.float32, torch.float16):
+            got, ref = _linear_w4_case(T, N, K, T * 7919 + N + K, out_dtype)
+            tol_check(got, ref, 1e-5 if out_dtype == torch.float32 else 2e-3)
+            u = np.uint16 if out_dtype == torch.float16 else np.uint32
+            assert np.array_equal(got.view(u), ref.view(u)), (pin, T, N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
 
 
 def test_linear_w4_extreme_accumulators():
@@ -239,8 +245,13 @@ def test_linear_w4_extreme_accumulators():
     s_a = np.ones(T, np.float32)
     y, acc = oracle.linear_w4(q, s_a, codes, s_w, np.float32)
     assert np.abs(acc).max() == 49 * K
-    gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), "int4", torch.float32)
-    assert np.array_equal(host(gy), y)
+    for pin in ("skinny", "gemv"):
+        qg.qift_debug_set_linear_path(pin)
+        try:
+            gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), "int4", torch.float32)
+        finally:
+            qg.qift_debug_set_linear_path("auto")
+        assert np.array_equal(host(gy), y), pin
 
 
 def test_linear_w4_unsupported_shapes_and_decode():

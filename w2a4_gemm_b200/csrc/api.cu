@@ -157,9 +157,19 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
         return QIFT_ERR_INVALID_ARG;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool f16 = out_dt == QIFT_F16;
-    if (set == QIFT_SET_INT4)  // one kernel family for 4-bit weights, whatever the debug pin
-        return from_cuda(qift::launch_linear_w4(q_act, act_scale, codes, w_scale, tokens, n_out, n_in, y, f16, s));
     int path = qift::debug_linear_path();
+    if (set == QIFT_SET_INT4) {
+        // 4-bit weights: the tensor-core skinny kernel for 2..16 tokens, the CUDA-core GEMV for one
+        // token; pinning "skinny" forces the former, any other pin the latter.
+        if (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))
+            return QIFT_ERR_UNSUPPORTED;
+        const bool skinny = path == qift::kPathSkinny ||
+                            (path == qift::kPathAuto && tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in));
+        if (skinny)
+            return from_cuda(qift::launch_linear_skinny(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
+                                                        n_in, y, f16, s));
+        return from_cuda(qift::launch_linear_w4(q_act, act_scale, codes, w_scale, tokens, n_out, n_in, y, f16, s));
+    }
     if (path == qift::kPathAuto) {
         if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
             path = qift::kPathGemmPair;

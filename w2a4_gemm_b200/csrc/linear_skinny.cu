@@ -23,6 +23,15 @@
 // k-slots 4q..4q+3 / 16+4q..16+4q+3 are (d[0], d[1]) in the first MMA and (d[2], d[3]) in the
 // second; the B fragment of token g comes from the same activation group w, permuted the same
 // way.  Every thread pairs A and B on identical k positions, so the dot products are exact.
+//
+// 4-bit weights (W4 = true; the Abstract's mixed W2/W4 layers).  A word holds 8 inputs as
+// two's-complement nibbles, byte i = inputs i (low) and i+4 (high), so (word << 4) & 0xF0F0F0F0
+// and word & 0xF0F0F0F0 are int8x4 registers holding 16 x the levels of inputs 0..3 and 4..7:
+// A fragments with no table and no permute.  Thread q's 16-byte load (4 words) covers two
+// activation groups of 16 inputs, j = 0, 1 (chunk c = 16 words = 128 inputs, group 8c + 2q + j);
+// the two words of group j give the k-slots (inputs 0..3, 4..7) of the first MMA and (8..11,
+// 12..15) of the second, against the activations in natural order.  The int32 sum is 16 x acc,
+// exactly (|16 acc| < 2^31 for n_in <= 32768); the epilogue shifts it right by 4.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -61,7 +70,7 @@ __device__ __forceinline__ void store_y<__half>(__half* p, float v) { *p = __flo
 // NT token tiles of 8 (T <= 8*NT).  KS: K slice per CTA in bytes (multiple of 256).  KSPLIT
 // warps share each 16-row group, taking alternate K chunks: 2 when the grid has at most one CTA
 // per SM (16 warps hide more latency), 1 otherwise (two CTAs of 8 warps fit on an SM).
-template <int NT, int KSPLIT, typename OutT>
+template <int NT, int KSPLIT, bool W4, typename OutT>
 __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const int8_t* __restrict__ q,
                                                             const float* __restrict__ s_a,
                                                             const uint32_t* __restrict__ codes,
@@ -82,9 +91,11 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, qd = lane & 3;
     const int row_block = blockIdx.x / C;
-    const int KW = K / 16;
-    const int kw0 = rank * (KS / 16);                  // first word of this CTA's slice
-    const int nchunks = KS / 256;
+    constexpr int CPW = W4 ? 8 : 16;                   // codes per word
+    constexpr int CHUNK_K = CHUNK_WORDS * CPW;         // inputs per chunk: 256, or 128 for W4
+    const int KW = K / CPW;
+    const int kw0 = rank * (KS / CPW);                 // first word of this CTA's slice
+    const int nchunks = KS / CHUNK_K;
     const int rw = warp % ROW_WARPS, ks = warp / ROW_WARPS;  // row warp, K parity
     const int my_n = (nchunks - ks + KSPLIT - 1) / KSPLIT;   // this warp's chunks: ks, ks+2, ...
     const int64_t r_lo = (int64_t)row_block * RB + rw * 16 + g;
@@ -117,7 +128,7 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
         for (int u = 0; u < 8; ++u) {
             const int i = i0 + u * THREADS + threadIdx.x;
             const int t = i / groups, G = i - t * groups;
-            const int64_t k = (int64_t)kw0 * 16 + (int64_t)G * 16;
+            const int64_t k = (int64_t)rank * KS + (int64_t)G * 16;  // input index of group G
             a[u] = make_uint4(0u, 0u, 0u, 0u);
             if (i < TP * groups && t < T && k + 16 <= K) a[u] = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
         }
@@ -126,9 +137,13 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
             const int i = i0 + u * THREADS + threadIdx.x;
             if (i < TP * groups) {
                 const int t = i / groups, G = i - t * groups;
-                uint32_t p[4];
-                permute_acts(a[u], p);
-                *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = make_uint4(p[0], p[1], p[2], p[3]);
+                uint4 v = a[u];
+                if constexpr (!W4) {
+                    uint32_t p[4];
+                    permute_acts(a[u], p);
+                    v = make_uint4(p[0], p[1], p[2], p[3]);
+                }
+                *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = v;
             }
         }
     }
@@ -153,6 +168,23 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
                 const uint32_t wl[4] = {buf[u][0].x, buf[u][0].y, buf[u][0].z, buf[u][0].w};
                 const uint32_t wh[4] = {buf[u][1].x, buf[u][1].y, buf[u][1].z, buf[u][1].w};
                 if (i + PF < my_n) load_chunk(c + KSPLIT * PF, buf[u][0], buf[u][1]);
+                if constexpr (W4) {
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        constexpr uint32_t M = 0xF0F0F0F0u;
+                        const uint32_t a1[4] = {(wl[2 * j] << 4) & M, (wh[2 * j] << 4) & M, wl[2 * j] & M, wh[2 * j] & M};
+                        const uint32_t a2[4] = {(wl[2 * j + 1] << 4) & M, (wh[2 * j + 1] << 4) & M, wl[2 * j + 1] & M,
+                                                wh[2 * j + 1] & M};
+                        const int slot = act_slot(c * (CHUNK_WORDS / 2) + 2 * qd + j);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
+                            mma_s8(acc[nt], a1, p.x, p.y);
+                            mma_s8(acc[nt], a2, p.z, p.w);
+                        }
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     uint32_t dl[4], dh[4];
@@ -206,6 +238,7 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
         const int t = i / rows_per, rl = rank * rows_per + (i - t * rows_per);
         int sum = 0;
         for (int p = 0; p < C; ++p) sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
+        if constexpr (W4) sum >>= 4;  // exact: every product was 16 x level x q
         const int64_t n = (int64_t)row_block * RB + rl;
         if (t < T && n < N) {
             const float v = __fmul_rn(__fmul_rn((float)sum, sw_s[rl]), sa_s[t]);
@@ -226,11 +259,11 @@ static int sm_count() {
     return cached[dev];
 }
 
-template <int NT, int KSPLIT, typename OutT>
+template <int NT, int KSPLIT, bool W4, typename OutT>
 static cudaError_t launch_k(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
                             int64_t T, int64_t N, int64_t K, int C, int KS, OutT* y, cudaStream_t s) {
     const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)NT * 8 * RBP * sizeof(int) + (size_t)(NT * 8 + RB) * 4;
-    cudaError_t e = ensure_smem(skinny_kernel<NT, KSPLIT, OutT>, smem);
+    cudaError_t e = ensure_smem(skinny_kernel<NT, KSPLIT, W4, OutT>, smem);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (N + RB - 1) / RB;
     cudaLaunchConfig_t cfg = {};
@@ -247,11 +280,11 @@ static cudaError_t launch_k(const int8_t* q, const float* s_a, const uint32_t* c
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, KSPLIT, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N, (int)K,
-                              KS, y);
+    return cudaLaunchKernelEx(&cfg, skinny_kernel<NT, KSPLIT, W4, OutT>, q, s_a, codes, s_w, lut, (int)T, (int)N,
+                              (int)K, KS, y);
 }
 
-template <int NT, typename OutT>
+template <int NT, bool W4, typename OutT>
 static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
                             int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
     // Cluster size: split K so that each CTA streams a slice of at most 2048 inputs (64 KB of
@@ -261,8 +294,8 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
     const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
     const int64_t ctas = ((N + RB - 1) / RB) * C;
-    if (ctas <= sm_count()) return launch_k<NT, 2, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
-    return launch_k<NT, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
+    if (ctas <= sm_count()) return launch_k<NT, 2, W4, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
+    return launch_k<NT, 1, W4, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
 }
 
 }  // namespace skinny
@@ -275,12 +308,20 @@ cudaError_t launch_linear_skinny(const int8_t* q, const float* s_a, const uint32
                                  int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
     if (T == 0 || N == 0) return cudaSuccess;
     const uint32_t lut = level_lut(set);
-    if (T <= 8) {
-        if (f16) return skinny::launch_t<1, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
-        return skinny::launch_t<1, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+    if (set == kSetInt4) {
+        if (T <= 8) {
+            if (f16) return skinny::launch_t<1, true, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+            return skinny::launch_t<1, true, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+        }
+        if (f16) return skinny::launch_t<2, true, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+        return skinny::launch_t<2, true, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
     }
-    if (f16) return skinny::launch_t<2, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
-    return skinny::launch_t<2, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+    if (T <= 8) {
+        if (f16) return skinny::launch_t<1, false, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+        return skinny::launch_t<1, false, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
+    }
+    if (f16) return skinny::launch_t<2, false, __half>(q, s_a, codes, s_w, lut, T, N, K, static_cast<__half*>(y), s);
+    return skinny::launch_t<2, false, float>(q, s_a, codes, s_w, lut, T, N, K, static_cast<float*>(y), s);
 }
 
 }  // namespace qift
