@@ -146,7 +146,8 @@ qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64
  *   codes     : u32 [n_out][n_in/16], w_scale: fp32 [n_out], from qift_quantize_weights.
  *   set       : QIFT_SET_QIFT or QIFT_SET_POT (QIFT_SET_STD -> QIFT_ERR_UNSUPPORTED), or
  *               QIFT_SET_INT4 (W4A4: codes u32 [n_out][n_in/8]; 1..16 tokens and n_in % 64 == 0,
- *               else QIFT_ERR_UNSUPPORTED; acc = sum q * level, on CUDA cores).
+ *               else QIFT_ERR_UNSUPPORTED; acc = sum q * level, |acc| <= 8*7*n_in; one token
+ *               on CUDA cores, 2..16 on the int8 tensor cores).
  *   y         : [tokens][n_out] out, out_dt QIFT_F32 or QIFT_F16 (round to nearest even).
  *   n_in      : multiple of 16, at most 32768 (so |acc| <= 7*4*n_in < 2^24 and (float)acc is
  *               exact).  tokens == 0 or n_out == 0 is a no-op.
@@ -173,7 +174,8 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
  *   x           : fp16 [tokens][n_in], 1 <= tokens <= 4; n_in % 64 == 0 and n_in <= 16384
  *                 (other valid sizes return QIFT_ERR_UNSUPPORTED: use the two calls).
  *   block       : Hadamard block as in qift_quantize_acts (0 = x already rotated).
- *   codes, w_scale, set (QIFT or POT), n_out, y, out_dt: as in qift_linear.
+ *   codes, w_scale, set (QIFT or POT; INT4 -> QIFT_ERR_UNSUPPORTED), n_out, y, out_dt: as in
+ *                 qift_linear.
  *   q_out       : int8 [tokens][n_in] or NULL -- receives the INT4 activations.
  *   act_scale_out: fp32 [tokens] or NULL -- receives s_a.
  * Like the decode GEMV it may read `codes` and `w_scale` before the kernel launched just before
