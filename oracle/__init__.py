@@ -15,7 +15,6 @@ Inference" (Huang, Tsai), Abstract.
 from __future__ import annotations
 
 import ctypes as C
-import os
 
 import numpy as np
 
@@ -47,6 +46,8 @@ def lib():
         L.qo_pack_int4.argtypes = [vp, i64, vp]
         L.qo_unpack_int4.argtypes = [vp, i64, vp]
         L.qo_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp]
+        L.qo_set_threads.argtypes = [C.c_int]
+        L.qo_set_threads.restype = C.c_int
         for name in ("qo_fwht_f64", "qo_rotate_f32", "qo_candidate_scales", "qo_quantize_weights",
                      "qo_unpack_codes", "qo_quantize_acts", "qo_linear", "qo_pack_int4", "qo_unpack_int4",
                      "qo_dequantize_kv", "qo_quantize_weights_w4", "qo_linear_w4"):
@@ -266,5 +267,9 @@ def pipeline(w: np.ndarray, x: np.ndarray, levelset, w_block: int, a_block: int,
 
 def threads() -> int:
     """Host threads the oracle's OpenMP loops use."""
-    v = os.environ.get("OMP_NUM_THREADS")
-    return int(v) if v else (os.cpu_count() or 1)
+    return int(lib().qo_set_threads(0))
+
+
+def set_threads(n: int) -> int:
+    """Run the oracle's loops on n host threads from now on; returns the count in force."""
+    return int(lib().qo_set_threads(int(n)))

@@ -24,6 +24,7 @@
  * Every function returns 0 on success and a negative number on a bad argument.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -481,4 +482,11 @@ int qo_linear(const int8_t* q, const float* s_a, const uint32_t* codes, const fl
         }
     }
     return overflow ? -3 : 0;
+}
+
+/* Host threads for the OpenMP loops above: n > 0 sets the count for later calls; returns the
+ * count now in force.  (Timing control only; no arithmetic depends on it.) */
+int qo_set_threads(int n) {
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
 }

@@ -57,3 +57,12 @@ def test_max_over_ranks_gloo_two_ranks():
 
 def test_max_over_ranks_single_process_is_identity():
     assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+def test_cpu_baseline_reports_all_cores_and_one_core():
+    import oracle
+    before = oracle.threads()
+    obj = bench.cpu_baseline_obj(bench.workload_def("single"), budget_s=0.2)
+    assert obj["kind"] == "oracle" and obj["cores"] == before and obj["value"] > 0
+    assert obj["single_core"]["cores"] == 1 and obj["single_core"]["value"] > 0
+    assert oracle.threads() == before  # the thread count is put back
