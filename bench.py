@@ -631,24 +631,37 @@ def run_offline(args, rank, world):
 
 
 def offline_cpu_baseline(budget_s=10.0):
-    """The oracle's rotate + quantize (three level sets) on a bounded sample of module rows."""
+    """The oracle's rotate + quantize (three level sets) on a bounded sample of module rows, on
+    every host core and then (a quarter of the budget) on one core."""
     import oracle
     from w2a4_gemm_b200 import synth
     rows = 16
     sample = [synth.weights(rows, n_in, (seed,)) for (_, _, _, n_in, seed) in synth.model_8b_modules()[:7]]
-    n, t0 = 0, time.perf_counter()
-    while True:
-        for w in sample:
-            wr = oracle.rotate_f32(w, synth.MODEL_8B_BLOCK)
-            for ls in ("qift", "pot", "std"):
-                oracle.quantize_weights(wr, ls)
-            n += 3 * w.size
-        if time.perf_counter() - t0 > budget_s:
-            break
-    secs = time.perf_counter() - t0
-    return {"value": n / secs, "unit": "weights/s", "cores": oracle.threads(), "kind": "oracle",
+
+    def rate(budget):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            for w in sample:
+                wr = oracle.rotate_f32(w, synth.MODEL_8B_BLOCK)
+                for ls in ("qift", "pot", "std"):
+                    oracle.quantize_weights(wr, ls)
+                n += 3 * w.size
+            if time.perf_counter() - t0 > budget:
+                break
+        secs = time.perf_counter() - t0
+        return n / secs, secs
+
+    all_cores = oracle.threads()
+    val, secs = rate(budget_s)
+    oracle.set_threads(1)
+    try:
+        val1, secs1 = rate(budget_s / 4)
+    finally:
+        oracle.set_threads(all_cores)
+    return {"value": val, "unit": "weights/s", "cores": all_cores, "kind": "oracle",
             "sample": f"{rows} rows of each of the 7 projections of one layer, 3 level sets, repeated for "
-                      f"{secs:.1f} s"}
+                      f"{secs:.1f} s",
+            "single_core": {"value": val1, "cores": 1, "sample": f"the same, repeated for {secs1:.1f} s"}}
 
 
 def main():
