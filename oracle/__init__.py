@@ -46,11 +46,14 @@ def lib():
         L.qo_pack_int4.argtypes = [vp, i64, vp]
         L.qo_unpack_int4.argtypes = [vp, i64, vp]
         L.qo_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp]
+        L.qo_quantize_weights_asym.argtypes = [vp, i64, i64, i32, f64, f64, vp, vp, vp, vp, vp]
+        L.qo_linear_asym.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp, vp]
         L.qo_set_threads.argtypes = [C.c_int]
         L.qo_set_threads.restype = C.c_int
         for name in ("qo_fwht_f64", "qo_rotate_f32", "qo_candidate_scales", "qo_quantize_weights",
                      "qo_unpack_codes", "qo_quantize_acts", "qo_linear", "qo_pack_int4", "qo_unpack_int4",
-                     "qo_dequantize_kv", "qo_quantize_weights_w4", "qo_linear_w4"):
+                     "qo_dequantize_kv", "qo_quantize_weights_w4", "qo_linear_w4", "qo_quantize_weights_asym",
+                     "qo_linear_asym"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -196,6 +199,41 @@ def linear_w4(q: np.ndarray, s_a: np.ndarray, codes: np.ndarray, s_w: np.ndarray
     acc = np.zeros((T, N), dtype=np.int32)
     y = np.zeros((T, N), dtype=np.float32)
     _check(lib().qo_linear_w4(_ptr(q), _ptr(s_a), _ptr(codes), _ptr(s_w), T, N, K, _ptr(acc), _ptr(y)), "linear_w4")
+    return y.astype(out_dtype), acc
+
+
+# ------------------------------------------------------------------- conventional asymmetric W2
+def quantize_weights_asym(w_rot: np.ndarray, grid_points: int = 100, lo: float = 0.2, hi: float = 1.0):
+    """Asymmetric 2-bit baseline: per channel scale s and integer zero point z in [0, 3], weight
+    (c - z) * s, range shrunk over the candidate grid.  Returns
+    ``(codes uint32 [N, K/16], scales f32 [N], zeros int32 [N], row_mse f64 [N], best_k int32 [N])``."""
+    w = np.ascontiguousarray(w_rot, dtype=np.float32)
+    n_out, n_in = w.shape
+    codes = np.zeros((n_out, n_in // 16), dtype=np.uint32)
+    scales = np.zeros(n_out, dtype=np.float32)
+    zeros = np.zeros(n_out, dtype=np.int32)
+    mse = np.zeros(n_out, dtype=np.float64)
+    best = np.zeros(n_out, dtype=np.int32)
+    _check(lib().qo_quantize_weights_asym(_ptr(w), n_out, n_in, grid_points, lo, hi, _ptr(codes), _ptr(scales),
+                                          _ptr(zeros), _ptr(mse), _ptr(best)), "quantize_weights_asym")
+    return codes, scales, zeros, mse, best
+
+
+def linear_asym(q: np.ndarray, s_a: np.ndarray, codes: np.ndarray, s_w: np.ndarray, zeros: np.ndarray,
+                out_dtype=np.float32):
+    """Asymmetric W2A4 linear: levels c - z per row, int32 accumulators, binary32 epilogue."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    zeros = np.ascontiguousarray(zeros, dtype=np.int32)
+    T, K = q.shape
+    N = codes.shape[0]
+    assert codes.shape[1] * 16 == K
+    acc = np.zeros((T, N), dtype=np.int32)
+    y = np.zeros((T, N), dtype=np.float32)
+    _check(lib().qo_linear_asym(_ptr(q), _ptr(s_a), _ptr(codes), _ptr(s_w), _ptr(zeros), T, N, K, _ptr(acc),
+                                _ptr(y)), "linear_asym")
     return y.astype(out_dtype), acc
 
 

@@ -363,6 +363,109 @@ int qo_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Conventional asymmetric W2 (the Abstract's comparison baseline, "Conventional asymmetric
+ * W2"): four uniform levels with a per-channel zero point.  The page gives no formula; the
+ * reading (R22) is the usual min-max affine quantizer with an integer zero point, searched
+ * over the same candidate grid as the other sets (R3) by shrinking the range:
+ *   lo_w = min(min_k w, 0), hi_w = max(max_k w, 0) (binary32; the range always holds 0);
+ *   candidate g: f_g as in R3; s_g = (float)((f_g * (hi_w - lo_w)) / 3) in binary64, one
+ *                rounding; z_g = nearest integer (ties to even) of -(f_g * lo_w) / s_g in
+ *                binary64, clamped to [0, 3] (0 when s_g = 0);
+ *   encode:      c = clamp(rint(w / s) + z, 0, 3), w / s one binary32 division, rint to
+ *                nearest even (c = z when s = 0);
+ *   error:       e = w - (float)(c - z) * s in binary32, e * e in binary32, summed in binary64
+ *                in index order (R9); smallest sum wins, the smaller g on ties (R4).
+ * The weight is (c - z) * s: code z is exactly 0.  Codes are packed as R10; the row keeps s and
+ * z.  The linear then reads the levels c - z: acc = sum q * (c - z) = sum q * c - z * sum q.
+ * ------------------------------------------------------------------------------------- */
+static int32_t asym_zero(double f, float lo_w, float s) {
+    if (!(s > 0.0f)) return 0;
+    double z = nearbyint(-(f * (double)lo_w) / (double)s);
+    return z < 0.0 ? 0 : (z > 3.0 ? 3 : (int32_t)z);
+}
+
+static int32_t encode_asym(float w, float s, int32_t z) {
+    if (!(s > 0.0f)) return z;
+    const float r = rintf(w / s);
+    const int32_t c = (int32_t)r + z;
+    return c < 0 ? 0 : (c > 3 ? 3 : c);
+}
+
+static float sq_err_asym(float w, float s, int32_t z, int32_t c) {
+    const float l = (float)(c - z) * s;
+    const float e = w - l;
+    return e * e;
+}
+
+int qo_quantize_weights_asym(const float* w, int64_t n_out, int64_t n_in, int32_t grid_points, double lo,
+                             double hi, uint32_t* codes, float* scales, int32_t* zeros, double* row_mse,
+                             int32_t* best_k) {
+    if (!w || !codes || !scales || !zeros || n_out < 0 || n_in <= 0 || (n_in % 16) != 0) return -1;
+    if (grid_points < 2 || grid_points > 4096) return -1;
+    const int64_t words = n_in / 16;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < n_out; ++n) {
+        const float* row = w + n * n_in;
+        float lo_w = 0.0f, hi_w = 0.0f;
+        for (int64_t k = 0; k < n_in; ++k) {
+            if (row[k] < lo_w) lo_w = row[k];
+            if (row[k] > hi_w) hi_w = row[k];
+        }
+        int32_t kbest = 0;
+        double best = 0.0;
+        for (int32_t g = 0; g < grid_points; ++g) {
+            const double f = lo + ((hi - lo) * (double)g) / (double)(grid_points - 1);
+            const float s = (float)((f * ((double)hi_w - (double)lo_w)) / 3.0);
+            const int32_t z = asym_zero(f, lo_w, s);
+            double acc = 0.0;
+            for (int64_t k = 0; k < n_in; ++k) acc += (double)sq_err_asym(row[k], s, z, encode_asym(row[k], s, z));
+            if (g == 0 || acc < best) {
+                best = acc;
+                kbest = g;
+            }
+        }
+        const double f = lo + ((hi - lo) * (double)kbest) / (double)(grid_points - 1);
+        const float s = (float)((f * ((double)hi_w - (double)lo_w)) / 3.0);
+        const int32_t z = asym_zero(f, lo_w, s);
+        uint32_t* out = codes + n * words;
+        for (int64_t j = 0; j < words; ++j) out[j] = 0u;
+        for (int64_t k = 0; k < n_in; ++k) out[k / 16] |= (uint32_t)encode_asym(row[k], s, z) << (2 * (k % 16));
+        scales[n] = s;
+        zeros[n] = z;
+        if (row_mse) row_mse[n] = best / (double)n_in;
+        if (best_k) best_k[n] = kbest;
+    }
+    return 0;
+}
+
+/* Asymmetric W2A4 linear: acc[t][n] = sum_k q[t][k] * (c[n][k] - z[n]) exactly (int64, must fit
+ * int32), then y = ((float)acc * s_w[n]) * s_a[t] (R13).  acc and y may be NULL. */
+int qo_linear_asym(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, const int32_t* zeros,
+                   int64_t tokens, int64_t n_out, int64_t n_in, int32_t* acc_out, float* y) {
+    if (!q || !s_a || !codes || !s_w || !zeros || tokens < 0 || n_out < 0 || n_in <= 0 || (n_in % 16) != 0)
+        return -1;
+    const int64_t words = n_in / 16;
+    int overflow = 0;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t t = 0; t < tokens; ++t) {
+        for (int64_t n = 0; n < n_out; ++n) {
+            int64_t sum = 0;
+            for (int64_t k = 0; k < n_in; ++k) {
+                const int32_t c = (int32_t)((codes[n * words + k / 16] >> (2 * (k % 16))) & 3u);
+                sum += (int64_t)q[t * n_in + k] * (int64_t)(c - zeros[n]);
+            }
+            if (sum > INT32_MAX || sum < INT32_MIN) {
+#pragma omp atomic write
+                overflow = 1;
+            }
+            if (acc_out) acc_out[t * n_out + n] = (int32_t)sum;
+            if (y) y[t * n_out + n] = ((float)sum * s_w[n]) * s_a[t];
+        }
+    }
+    return overflow ? -3 : 0;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Symmetric per-token INT4 activation quantization (the "A4" of W2A4 in the Abstract).
  * Input: the rotated activations after their single rounding to binary16, given here as
  * the binary32 values of those binary16 numbers.
