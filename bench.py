@@ -538,6 +538,29 @@ def alu_peak_evals(sm_mhz=1965.0, sms=148):
     return sms * 4 * 32 * sm_mhz * 1e6 / ALU_EVAL_INSTR
 
 
+def excess_kurtosis(x) -> float:
+    """Excess kurtosis E[(x - mean)^4] / var^2 - 3 of all entries of a tensor, in float64 (0 for a
+    Gaussian; the Hadamard rotation should bring heavy-tailed rows towards it)."""
+    d = x.double().flatten()
+    d = d - d.mean()
+    v = (d * d).mean()
+    return float((d ** 4).mean() / (v * v) - 3.0)
+
+
+def per_projection_mse(mods, row_mse_by_set):
+    """Reconstruction MSE per projection name over all layers: {set: {proj: mse}}.  row_mse_by_set
+    maps a set to one array of per-row MSEs per module, aligned with `mods` (layer, proj, n_out,
+    n_in, seed)."""
+    out = {}
+    for ls, per_mod in row_mse_by_set.items():
+        num, den = {}, {}
+        for (_, proj, n_out, n_in, _), m in zip(mods, per_mod):
+            num[proj] = num.get(proj, 0.0) + float(np.asarray(m, dtype=np.float64).sum()) * n_in
+            den[proj] = den.get(proj, 0) + n_out * n_in
+        out[ls] = {p: num[p] / den[p] for p in num}
+    return out
+
+
 def run_offline(args, rank, world):
     import torch
     import w2a4_gemm_b200 as qg
@@ -587,6 +610,16 @@ def run_offline(args, rank, world):
     n_w = sum(w.numel() for w in W)
     value = world * 3 * n_w * args.steps / secs
     set_mse = {ls: float(sum((m * w.shape[1]).sum().item() for m, w in zip(mse[ls], W)) / n_w) for ls in mse}
+    proj_mse = per_projection_mse(mods, {ls: [m.cpu().numpy() for m in mse[ls]] for ls in mse})
+    # Kurtosis of layer 0's projections before and after the rotation (a diagnostic of the
+    # Gaussianisation the rotation is there for), outside the timed region.
+    kurt = {}
+    for j, (layer, proj, n_out, n_in, _) in enumerate(mods):
+        if layer != 0:
+            break
+        r = rot[: W[j].numel()].view(n_out, n_in)
+        qg.qift_rotate(W[j], synth.MODEL_8B_BLOCK, out=r)
+        kurt[proj] = {"before": excess_kurtosis(W[j]), "after": excess_kurtosis(r)}
 
     # Live per-kernel timing of the two offline kernels on the largest module.
     wbig = max(W, key=lambda w: w.numel())
@@ -613,7 +646,8 @@ def run_offline(args, rank, world):
                                   "level sets; Student-t(4)*0.02 weights drawn on the device",
                    "weights": n_w, "level_sets": ["qift", "pot", "std"], "grid_points": 100,
                    "l2": "inputs larger than L2 (27.9 GB of fp32 weights)",
-                   "reconstruction_mse": set_mse,
+                   "reconstruction_mse": set_mse, "reconstruction_mse_per_projection": proj_mse,
+                   "excess_kurtosis_layer0": kurt,
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "roofline": {"bound": "alu", "achieved": evals / 1e12, "peak": peak / 1e12, "unit": "T candidate-evals/s",
                      "frac": evals / peak, "traffic": profiled_traffic("offline"),

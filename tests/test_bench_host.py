@@ -66,3 +66,21 @@ def test_cpu_baseline_reports_all_cores_and_one_core():
     assert obj["kind"] == "oracle" and obj["cores"] == before and obj["value"] > 0
     assert obj["single_core"]["cores"] == 1 and obj["single_core"]["value"] > 0
     assert oracle.threads() == before  # the thread count is put back
+
+
+def test_excess_kurtosis_known_values():
+    import numpy as np
+    import torch
+    assert bench.excess_kurtosis(torch.tensor([-1.0, 1.0, -1.0, 1.0])) == -2.0   # two-point law
+    g = torch.from_numpy(np.random.default_rng(0).normal(size=400_000))
+    assert abs(bench.excess_kurtosis(g)) < 0.05                                   # Gaussian: 0
+    t = torch.from_numpy(np.random.default_rng(1).standard_t(6, size=400_000))
+    assert 2.0 < bench.excess_kurtosis(t) < 4.5                                   # t(6): 6/(6-4) = 3
+
+
+def test_per_projection_mse_weights_modules_by_size():
+    mods = [(0, "q", 2, 4, 0), (0, "down", 1, 8, 1), (1, "q", 1, 4, 2)]
+    rows = {"qift": [[1.0, 3.0], [5.0], [8.0]]}
+    got = bench.per_projection_mse(mods, rows)["qift"]
+    # q: (1 + 3) * 4 + 8 * 4 over 3 rows of 4 -> 48 / 12; down: 5 * 8 / 8
+    assert got == {"q": 4.0, "down": 5.0}
