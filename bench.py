@@ -216,6 +216,24 @@ class OursState:
         return sum(1 + int(L["quant"]) for L in self.layers)
 
 
+def library_int8_tops(torch, n=8192, reps=10):
+    """Dense int8 TOPS of the vendor library GEMM (torch._int_mm, int8 x int8 -> int32) on an
+    n x n x n problem: the best of `reps` launches, each timed with CUDA events."""
+    a = torch.randint(-7, 8, (n, n), dtype=torch.int8, device="cuda")
+    b = torch.randint(-7, 8, (n, n), dtype=torch.int8, device="cuda")
+    for _ in range(3):
+        torch._int_mm(a, b)
+    best = float("inf")
+    for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch._int_mm(a, b)
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e) / 1e3)
+    return 2.0 * n ** 3 / best / 1e12
+
+
 def max_over_ranks(value: float, world: int) -> float:
     """The largest of every rank's value (one all-reduce); the value itself on one rank."""
     if world <= 1:
@@ -357,6 +375,13 @@ def run_ours(args, rank, world):
                 "frac": ach / pk["int8_tops"], "traffic": profiled_traffic(args.workload),
                 "kernel": "qift_linear (GEMM)",
                 "peak_source": pk["source"] + " bf16 burst x 2 (int8 nominal ratio)"}
+        # A second reference, for context only: the vendor library's int8 GEMM on this GPU.
+        try:
+            lib_tops = library_int8_tops(torch)
+            roof["library_int8"] = {"tops": lib_tops, "frac": ach / lib_tops,
+                                    "what": "torch._int_mm (the vendor int8 GEMM) at 8192^3, best of 10, same run"}
+        except RuntimeError as e:  # an int8 GEMM the installed library does not offer on this GPU
+            roof["library_int8"] = {"tops": None, "error": str(e).splitlines()[0][:200]}
 
     # End to end through the public API: every step copies its x from pinned host memory to the
     # device, runs the calls and copies y back to pinned host memory.  As in a serving loop the
