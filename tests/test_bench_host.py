@@ -1,5 +1,6 @@
-"""Host-side pieces of bench.py: algorithmic byte counts and the max-over-ranks timing
-reduction, the latter with two gloo ranks on the CPU (the N-GPU replica path)."""
+"""Host-side pieces of bench.py: algorithmic byte counts, the max-over-ranks timing reduction
+with two gloo ranks on the CPU (the N-GPU replica path), the CPU-oracle baselines and their
+diagnostics, and the reference arm launched under torchrun."""
 import os
 import socket
 
@@ -84,3 +85,22 @@ def test_per_projection_mse_weights_modules_by_size():
     got = bench.per_projection_mse(mods, rows)["qift"]
     # q: (1 + 3) * 4 + 8 * 4 over 3 rows of 4 -> 48 / 12; down: 5 * 8 / 8
     assert got == {"q": 4.0, "down": 5.0}
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
+    # Launched the way the multi-GPU runs are (one process per rank): rank 0 alone times the
+    # oracle and prints; the other rank exits 0 without work.
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--workload", "single", "--steps", "2", "--warmup", "1"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
