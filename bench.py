@@ -635,7 +635,23 @@ def run_offline(args, rank, world):
     n_w = sum(w.numel() for w in W)
     value = world * 3 * n_w * args.steps / secs
     set_mse = {ls: float(sum((m * w.shape[1]).sum().item() for m, w in zip(mse[ls], W)) / n_w) for ls in mse}
-    proj_mse = per_projection_mse(mods, {ls: [m.cpu().numpy() for m in mse[ls]] for ls in mse})
+    # The comparison baseline the page names (conventional asymmetric W2), outside the timed
+    # region: the same rotation and candidate grid, with a per-row zero point.
+    zeros = torch.empty(max(w.shape[0] for w in W), dtype=torch.int32, device=dev)
+    asym_rows = []
+    for w in W:
+        n_out, n_in = w.shape
+        r = rot[: w.numel()].view(n_out, n_in)
+        qg.qift_rotate(w, synth.MODEL_8B_BLOCK, out=r)
+        m_asym = torch.empty(n_out, dtype=torch.float64, device=dev)
+        qg._check(L.qift_quantize_weights_asym(qg._ptr(r), n_out, n_in, 100, 0.2, 1.0, qg._ptr(codes),
+                                               qg._ptr(scales), qg._ptr(zeros), qg._ptr(m_asym),
+                                               qg._stream(None)), "qift_quantize_weights_asym")
+        asym_rows.append(m_asym.cpu().numpy())
+    set_mse["asym"] = float(sum(float(m.sum()) * w.shape[1] for m, w in zip(asym_rows, W)) / n_w)
+    rows_by_set = {ls: [m.cpu().numpy() for m in mse[ls]] for ls in mse}
+    rows_by_set["asym"] = asym_rows
+    proj_mse = per_projection_mse(mods, rows_by_set)
     # Kurtosis of layer 0's projections before and after the rotation (a diagnostic of the
     # Gaussianisation the rotation is there for), outside the timed region.
     kurt = {}
@@ -670,6 +686,7 @@ def run_offline(args, rank, world):
                                   "linear modules of an 8B-shaped model, for each of the Qift, PoT and standard "
                                   "level sets; Student-t(4)*0.02 weights drawn on the device",
                    "weights": n_w, "level_sets": ["qift", "pot", "std"], "grid_points": 100,
+                   "mse_baseline": "asym: conventional asymmetric W2 (scale + zero point), not timed",
                    "l2": "inputs larger than L2 (27.9 GB of fp32 weights)",
                    "reconstruction_mse": set_mse, "reconstruction_mse_per_projection": proj_mse,
                    "excess_kurtosis_layer0": kurt,

@@ -105,6 +105,26 @@ qift_status qift_rotate_quantize_weights(const float* w, int64_t n_out, int64_t 
                                          uint32_t* codes, float* scales, double* row_mse, void* stream);
 
 /*
+ * qift_quantize_weights_asym -- the conventional asymmetric W2 baseline the Abstract compares the
+ * no-zero sets against ("Conventional asymmetric W2"): per output channel a scale s and an
+ * integer zero point z in [0, 3], weight (c - z) * s.  The page gives no formula; this is the
+ * min-max affine quantizer with the range shrunk over the same candidate grid:
+ *   candidate f (as in qift_quantize_weights): s = (f * (max(max w, 0) - min(min w, 0))) / 3 in
+ *   binary64, one rounding to binary32; z = the nearest integer, ties to even, of
+ *   -(f * min(min w, 0)) / s in binary64, clamped to [0, 3] (0 when s = 0);
+ *   code c = clamp(rint(w / s) + z, 0, 3), w / s one binary32 division (c = z when s = 0);
+ *   error e = w - (c - z) * s in binary32, e * e summed in binary64 in input order; the
+ *   smallest sum wins, the earlier candidate on ties.
+ *   w_rot, n_out, n_in, grid_points, lo, hi, codes (2-bit, packed as in qift_quantize_weights),
+ *   row_mse, stream: as in qift_quantize_weights.
+ *   scales : fp32 [n_out] out: s.        zeros : int32 [n_out] out: z (4-byte aligned).
+ * The library has no linear for this set: it serves the reconstruction-error comparison.
+ */
+qift_status qift_quantize_weights_asym(const float* w_rot, int64_t n_out, int64_t n_in, int32_t grid_points,
+                                       double lo, double hi, uint32_t* codes, float* scales, int32_t* zeros,
+                                       double* row_mse, void* stream);
+
+/*
  * qift_quantize_acts -- optional rotation + symmetric per-token INT4 quantization.
  * Abstract: the "A4" of rotated W2A4 inference.
  *   x      : fp16 (binary16 bits) [tokens][n_in], n_in % 16 == 0, n_in <= 32768.

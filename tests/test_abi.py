@@ -79,6 +79,18 @@ def test_quantize_weights_validation(L):
     assert f(None, 0, 64, 0, 100, 0.2, 1.0, None, None, None, None) == q.QIFT_OK
 
 
+def test_quantize_weights_asym_validation(L):
+    bad = q.QIFT_ERR_INVALID_ARG
+    f = L.qift_quantize_weights_asym
+    assert f(FAKE, 4, 40, 100, 0.2, 1.0, FAKE, FAKE, FAKE, None, None) == bad    # n_in % 16
+    assert f(FAKE, 4, 64, 1, 0.2, 1.0, FAKE, FAKE, FAKE, None, None) == bad      # grid
+    assert f(FAKE, 4, 64, 100, 0.5, 0.4, FAKE, FAKE, FAKE, None, None) == bad    # hi < lo
+    assert f(FAKE, 4, 64, 100, 0.2, 1.0, FAKE, FAKE, None, None, None) == bad    # null zeros
+    assert f(FAKE, 4, 64, 100, 0.2, 1.0, FAKE, FAKE, C.c_void_p(0x10002), None, None) == bad  # zeros alignment
+    assert f(FAKE, 4, 65536, 100, 0.2, 1.0, FAKE, FAKE, FAKE, None, None) == q.QIFT_ERR_UNSUPPORTED
+    assert f(None, 0, 64, 100, 0.2, 1.0, None, None, None, None, None) == q.QIFT_OK
+
+
 def test_quantize_acts_validation(L):
     bad = q.QIFT_ERR_INVALID_ARG
     f = L.qift_quantize_acts

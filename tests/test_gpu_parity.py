@@ -166,6 +166,42 @@ def test_rotate_quantize_weights_block0_and_bad_block():
             qg.qift_rotate_quantize_weights(dev(w), bad, "qift")
 
 
+# ------------------------------------------------------- conventional asymmetric W2 baseline
+@pytest.mark.parametrize("n_out,n_in,block", [(5, 16, 16), (33, 48, 16), (64, 512, 128), (40, 4096, 4096),
+                                               (9, 11008, 128), (7, 3072, 128)])
+def test_quantize_weights_asym_parity(n_out, n_in, block):
+    w = oracle.rotate_f32(synth.weights(n_out, n_in, (n_in, 29)), block)
+    codes, scales, zeros, mse, _ = oracle.quantize_weights_asym(w)
+    gc, gs, gz, gm = qg.qift_quantize_weights_asym(dev(w))
+    assert np.array_equal(codes_u32(gc), codes)
+    assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+    assert np.array_equal(host(gz), zeros)
+    assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
+def test_quantize_weights_asym_edge_rows():
+    # zero row, rows on one side of 0, a lossless grid row, a tie of the zero point, signed zeros
+    K = 64
+    w = np.zeros((7, K), np.float32)
+    w[1] = np.linspace(0.5, 3.0, K, dtype=np.float32)
+    w[2] = np.linspace(-3.0, -0.5, K, dtype=np.float32)
+    rng = np.random.default_rng(5)
+    c = rng.integers(0, 4, size=K)
+    c[0], c[1] = 0, 3
+    w[3] = ((c - 1) * 0.25).astype(np.float32)
+    w[4] = np.linspace(-1.5, 1.5, K, dtype=np.float32)
+    w[5, :] = -0.0
+    w[5, 3] = 0.5
+    w[6] = synth.weights(1, K, (97,))[0]
+    for grid, lo, hi in ((100, 0.2, 1.0), (2, 1.0, 1.0), (256, 0.05, 4.0)):
+        codes, scales, zeros, mse, _ = oracle.quantize_weights_asym(w, grid, lo, hi)
+        gc, gs, gz, gm = qg.qift_quantize_weights_asym(dev(w), grid, lo, hi)
+        assert np.array_equal(codes_u32(gc), codes), grid
+        assert np.array_equal(host(gs).view(np.uint32), scales.view(np.uint32))
+        assert np.array_equal(host(gz), zeros)
+        assert np.array_equal(host(gm).view(np.uint64), mse.view(np.uint64))
+
+
 # ----------------------------------------------------------------- W4A4 (4-bit weights)
 @pytest.mark.parametrize("n_out,n_in,block", [(5, 16, 16), (33, 48, 16), (64, 512, 128), (40, 4096, 4096),
                                                (9, 11008, 128), (7, 3072, 128)])

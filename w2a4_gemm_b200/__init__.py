@@ -45,6 +45,7 @@ def lib() -> C.CDLL:
         L.qift_rotate.argtypes = [vp, vp, i32, i64, i64, i32, vp]
         L.qift_quantize_weights.argtypes = [vp, i64, i64, i32, i32, f64, f64, vp, vp, vp, vp]
         L.qift_rotate_quantize_weights.argtypes = [vp, i64, i64, i32, i32, i32, f64, f64, vp, vp, vp, vp]
+        L.qift_quantize_weights_asym.argtypes = [vp, i64, i64, i32, f64, f64, vp, vp, vp, vp, vp]
         L.qift_quantize_acts.argtypes = [vp, i64, i64, i32, vp, vp, vp]
         L.qift_quantize_kv.argtypes = [vp, i64, i64, i32, vp, vp, vp]
         L.qift_dequantize_kv.argtypes = [vp, vp, i64, i64, i32, vp, vp]
@@ -58,7 +59,8 @@ def lib() -> C.CDLL:
         L.qift_debug_set_pdl.argtypes = [i32]
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
-        for name in ("qift_rotate", "qift_quantize_weights", "qift_rotate_quantize_weights", "qift_quantize_acts",
+        for name in ("qift_rotate", "qift_quantize_weights", "qift_rotate_quantize_weights",
+                     "qift_quantize_weights_asym", "qift_quantize_acts",
                      "qift_quantize_kv", "qift_dequantize_kv",
                      "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
@@ -137,6 +139,26 @@ def qift_quantize_weights(w_rot: torch.Tensor, levelset="qift", grid_points: int
                                        _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
            "qift_quantize_weights")
     return codes, scales, mse
+
+
+def qift_quantize_weights_asym(w_rot: torch.Tensor, grid_points: int = 100, lo: float = 0.2, hi: float = 1.0,
+                               with_mse: bool = True, stream=None):
+    """Conventional asymmetric W2 baseline: per-row scale and integer zero point, weight (c - z) * s.
+
+    Returns ``(codes int32-viewed-as-u32 [N, K/16], scales f32 [N], zeros int32 [N],
+    row_mse f64 [N] or None)``.
+    """
+    _cuda(w_rot, "w_rot", torch.float32)
+    n_out, n_in = w_rot.shape
+    dev = w_rot.device
+    codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
+    scales = torch.empty(n_out, dtype=torch.float32, device=dev)
+    zeros = torch.empty(n_out, dtype=torch.int32, device=dev)
+    mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
+    _check(lib().qift_quantize_weights_asym(_ptr(w_rot), n_out, n_in, grid_points, lo, hi, _ptr(codes),
+                                            _ptr(scales), _ptr(zeros), _ptr(mse), _stream(stream)),
+           "qift_quantize_weights_asym")
+    return codes, scales, zeros, mse
 
 
 def qift_rotate_quantize_weights(w: torch.Tensor, block: int, levelset="qift", grid_points: int = 100,

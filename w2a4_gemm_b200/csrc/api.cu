@@ -85,6 +85,23 @@ qift_status qift_quantize_weights(const float* w_rot, int64_t n_out, int64_t n_i
                                                    row_mse, static_cast<cudaStream_t>(stream)));
 }
 
+qift_status qift_quantize_weights_asym(const float* w_rot, int64_t n_out, int64_t n_in, int32_t grid_points,
+                                       double lo, double hi, uint32_t* codes, float* scales, int32_t* zeros,
+                                       double* row_mse, void* stream) {
+    if (n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
+    if (grid_points < 2 || grid_points > 256) return QIFT_ERR_INVALID_ARG;
+    if (!(lo > 0.0) || !(hi >= lo) || !(hi <= 4.0)) return QIFT_ERR_INVALID_ARG;
+    if (n_in > kMaxInner) return QIFT_ERR_UNSUPPORTED;
+    if (n_out == 0) return QIFT_OK;
+    if (!w_rot || !codes || !scales || !zeros || !aligned16(w_rot) || !aligned16(codes) || !aligned4(scales) ||
+        !aligned4(zeros))
+        return QIFT_ERR_INVALID_ARG;
+    if (row_mse && !aligned8(row_mse)) return QIFT_ERR_INVALID_ARG;
+    if (n_out > 0x7fffffff) return QIFT_ERR_UNSUPPORTED;
+    return from_cuda(qift::launch_quantize_weights_asym(w_rot, n_out, n_in, grid_points, lo, hi, codes, scales, zeros,
+                                                        row_mse, static_cast<cudaStream_t>(stream)));
+}
+
 qift_status qift_rotate_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int32_t block,
                                          qift_levelset set, int32_t grid_points, double lo, double hi,
                                          uint32_t* codes, float* scales, double* row_mse, void* stream) {

@@ -15,6 +15,7 @@ constexpr int kSetQift = 0;
 constexpr int kSetPot = 1;
 constexpr int kSetStd = 2;
 constexpr int kSetInt4 = 3;  // 4-bit weights {-7..7} * s as two's-complement nibbles, eight per word
+constexpr int kSetAsym = 4;  // conventional asymmetric W2: (c - z) * s, integer zero point z per row
 
 // Integer level table of a set packed as four signed bytes, byte c = level of code c, so that
 // one byte permute (prmt) turns four 2-bit codes into four int8 weights.

@@ -52,6 +52,10 @@ cudaError_t launch_dequantize_kv(const uint8_t* packed, const float* scales, int
 cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in, int set, int grid_points,
                                     double lo, double hi, uint32_t* codes, float* scales, double* row_mse,
                                     cudaStream_t s, int block = 0);
+// The asymmetric W2 baseline: the same search with a per-row zero point (zeros: int32 [n_out]).
+cudaError_t launch_quantize_weights_asym(const float* w, int64_t n_out, int64_t n_in, int grid_points, double lo,
+                                         double hi, uint32_t* codes, float* scales, int32_t* zeros, double* row_mse,
+                                         cudaStream_t s);
 
 // Decode-size linear: HBM-streaming GEMV (CUDA-core dp4a).
 cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,

@@ -28,8 +28,11 @@ template <int SET>
 struct Encoder {
     float s, thr1, thr2, l_in, l_out;
     float thr[7];  // W4: midpoints (j + 0.5) s rounded down, j = 0..6
-    __device__ __forceinline__ explicit Encoder(float s_) : s(s_) {
-        if constexpr (SET == kSetInt4) {        // levels {-7..7} s; midpoints (j + 0.5) s
+    int z;         // asymmetric: the zero point
+    __device__ __forceinline__ explicit Encoder(float s_, int z_ = 0) : s(s_), z(z_) {
+        if constexpr (SET == kSetAsym) {
+            // (c - z) * s: nothing to precompute; the code comes from one IEEE division
+        } else if constexpr (SET == kSetInt4) {        // levels {-7..7} s; midpoints (j + 0.5) s
 #pragma unroll
             for (int j = 0; j < 7; ++j) thr[j] = __fmul_rd((float)j + 0.5f, s);
         } else if constexpr (SET == kSetQift) {  // levels +-0.5 s, +-1.5 s; midpoint s
@@ -55,7 +58,11 @@ struct Encoder {
     // Code: 0..3 in increasing level order, or (W4) the level's two's-complement nibble.  Ties go
     // to the smaller magnitude; w >= 0 is positive.
     __device__ __forceinline__ uint32_t code(float w) const {
-        if constexpr (SET == kSetInt4) {
+        if constexpr (SET == kSetAsym) {  // clamp(rint(w / s) + z, 0, 3); c = z when s = 0
+            if (!(s > 0.0f)) return (uint32_t)z;
+            const int c = (int)rintf(__fdiv_rn(w, s)) + z;
+            return (uint32_t)(c < 0 ? 0 : (c > 3 ? 3 : c));
+        } else if constexpr (SET == kSetInt4) {
             const int j = w4_mag(fabsf(w));
             return (uint32_t)(w >= 0.0f ? j : -j) & 0xFu;
         } else if constexpr (SET == kSetStd) {
@@ -72,7 +79,9 @@ struct Encoder {
     // Squared reconstruction error of w, in fp32, for its code.
     __device__ __forceinline__ float sq_err(float w) const {
         float e;
-        if constexpr (SET == kSetInt4) {
+        if constexpr (SET == kSetAsym) {
+            e = __fsub_rn(w, __fmul_rn((float)((int)code(w) - z), s));
+        } else if constexpr (SET == kSetInt4) {
             const float a = fabsf(w);
             // (float)j by the exact magic-number add (j <= 7), off the conversion unit
             const float jf = __fsub_rn(__int_as_float(0x4B400000 + w4_mag(a)), 12582912.0f);
@@ -169,11 +178,14 @@ template <int SET, bool ROT>
 __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __restrict__ w, int64_t n_out, int64_t K,
                                                              int R, int G, double lo, double hi,
                                                              uint32_t* __restrict__ codes, float* __restrict__ scales,
-                                                             double* __restrict__ row_mse, int logb, float c) {
+                                                             int32_t* __restrict__ zeros, double* __restrict__ row_mse,
+                                                             int logb, float c) {
     extern __shared__ __align__(16) float ws[];  // R rows of K floats
     __shared__ float cand[kQwMaxRows * kQwMaxG];
     __shared__ double mse[kQwMaxRows * kQwMaxG];
     __shared__ float red[kQwMaxRows][32];
+    __shared__ float red_lo[kQwMaxRows][32];    // asymmetric: min(w, 0) partials
+    __shared__ int8_t zc[kQwMaxRows * kQwMaxG];  // asymmetric: each candidate's zero point
     __shared__ int best_s[kQwMaxRows];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x, nwarps = nthr >> 5;
     const int64_t row0 = (int64_t)blockIdx.x * R;
@@ -189,10 +201,12 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
         __syncthreads();
         fwht_rows_in_smem(ws, rows, (int)K, logb, c);
     }
-    float m[kQwMaxRows];
+    // (Asymmetric set: the row's max(w, 0) in m and min(w, 0) in mn instead.)
+    float m[kQwMaxRows], mn[kQwMaxRows];
 #pragma unroll
     for (int r = 0; r < kQwMaxRows; ++r) {
         m[r] = 0.0f;
+        mn[r] = 0.0f;
         if (r < rows) {
             const float* wr = w + (row0 + r) * K;
             for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4) {
@@ -203,34 +217,63 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
                     v = *reinterpret_cast<const float4*>(wr + i);
                     *reinterpret_cast<float4*>(ws + r * K + i) = v;
                 }
-                m[r] = fmaxf(m[r], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                if constexpr (SET == kSetAsym) {
+                    m[r] = fmaxf(m[r], fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+                    mn[r] = fminf(mn[r], fminf(fminf(v.x, v.y), fminf(v.z, v.w)));
+                } else {
+                    m[r] = fmaxf(m[r], fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                }
             }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m[r] = fmaxf(m[r], __shfl_xor_sync(0xffffffffu, m[r], o));
-        if (lane == 0) red[r][warp] = m[r];
+        for (int o = 16; o > 0; o >>= 1) {
+            m[r] = fmaxf(m[r], __shfl_xor_sync(0xffffffffu, m[r], o));
+            if constexpr (SET == kSetAsym) mn[r] = fminf(mn[r], __shfl_xor_sync(0xffffffffu, mn[r], o));
+        }
+        if (lane == 0) {
+            red[r][warp] = m[r];
+            red_lo[r][warp] = mn[r];
+        }
     }
     __syncthreads();
     if (tid < kQwMaxRows) {
-        float v = 0.0f;
-        for (int i = 0; i < nwarps; ++i) v = fmaxf(v, red[tid][i]);
+        float v = 0.0f, u = 0.0f;
+        for (int i = 0; i < nwarps; ++i) {
+            v = fmaxf(v, red[tid][i]);
+            u = fminf(u, red_lo[tid][i]);
+        }
         red[tid][0] = v;
+        red_lo[tid][0] = u;
     }
     __syncthreads();
 
     // Candidate scales, binary64 in the order lo + ((hi - lo) * k) / (G - 1), then * m / L.
+    // Asymmetric set: s = (f * (max - min)) / 3, and the zero point z = rint(-(f * min) / s),
+    // ties to even, clamped to [0, 3] (0 when s = 0).
     const double lambda = SET == kSetQift ? 1.5 : (SET == kSetPot ? 4.0 : (SET == kSetInt4 ? 7.0 : 2.0));
     for (int f = tid; f < rows * G; f += nthr) {
         const int r = f / G, g = f - r * G;
         const double fr = __dadd_rn(lo, __ddiv_rn(__dmul_rn(__dsub_rn(hi, lo), (double)g), (double)(G - 1)));
-        cand[r * kQwMaxG + g] = __double2float_rn(__ddiv_rn(__dmul_rn(fr, (double)red[r][0]), lambda));
+        if constexpr (SET == kSetAsym) {
+            const double range = __dsub_rn((double)red[r][0], (double)red_lo[r][0]);
+            const float sv = __double2float_rn(__ddiv_rn(__dmul_rn(fr, range), 3.0));
+            int z = 0;
+            if (sv > 0.0f) {
+                z = __double2int_rn(__ddiv_rn(-__dmul_rn(fr, (double)red_lo[r][0]), (double)sv));
+                z = z < 0 ? 0 : (z > 3 ? 3 : z);
+            }
+            cand[r * kQwMaxG + g] = sv;
+            zc[r * kQwMaxG + g] = (int8_t)z;
+        } else {
+            cand[r * kQwMaxG + g] = __double2float_rn(__ddiv_rn(__dmul_rn(fr, (double)red[r][0]), lambda));
+        }
     }
     __syncthreads();
 
     // MSE of every (row, candidate): sequential over the row, fp32 squared error widened to fp64.
     for (int f = tid; f < rows * G; f += nthr) {
         const int r = f / G, g = f - r * G;
-        const Encoder<SET> enc(cand[r * kQwMaxG + g]);
+        const Encoder<SET> enc(cand[r * kQwMaxG + g], SET == kSetAsym ? (int)zc[r * kQwMaxG + g] : 0);
         double acc = 0.0;
         const float4* w4 = reinterpret_cast<const float4*>(ws + r * K);
         for (int64_t i = 0; i < K / 4; ++i) {
@@ -263,7 +306,7 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
     for (int r = 0; r < rows; ++r) {
         const int b = best_s[r];
         const float sr = cand[r * kQwMaxG + b];
-        const Encoder<SET> enc(sr);
+        const Encoder<SET> enc(sr, SET == kSetAsym ? (int)zc[r * kQwMaxG + b] : 0);
         uint32_t* crow = codes + (row0 + r) * (K / CPW);
         for (int64_t j = tid; j < K / CPW; j += nthr) {
             const float4* w4 = reinterpret_cast<const float4*>(ws + r * K + j * CPW);
@@ -280,6 +323,7 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
         }
         if (tid == 0) {
             scales[row0 + r] = SET == kSetQift ? __fmul_rn(sr, 0.5f) : sr;
+            if constexpr (SET == kSetAsym) zeros[row0 + r] = zc[r * kQwMaxG + b];
             if (row_mse) row_mse[row0 + r] = __ddiv_rn(mse[r * kQwMaxG + b], (double)K);
         }
     }
@@ -287,7 +331,8 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
 
 template <int SET>
 static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
-                             uint32_t* codes, float* scales, double* row_mse, int block, cudaStream_t s) {
+                             uint32_t* codes, float* scales, int32_t* zeros, double* row_mse, int block,
+                             cudaStream_t s) {
     // As many rows per CTA as fit in ~100 KB of shared memory (so several CTAs share an SM).
     int R = (int)std::min<int64_t>(kQwMaxRows, std::max<int64_t>(1, (100 * 1024) / (n_in * 4)));
     const int threads = std::max(128, std::min(1024, (R * G + 31) / 32 * 32));
@@ -299,13 +344,13 @@ static cudaError_t launch_qw(const float* w, int64_t n_out, int64_t n_in, int G,
         // Normalisation constant as in qift_rotate: binary64 1/sqrt(b) rounded once to binary32.
         const float c = (float)(1.0 / sqrt((double)block));
         quant_weights_kernel<SET, true><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes,
-                                                                              scales, row_mse, ilog2(block), c);
+                                                                              scales, zeros, row_mse, ilog2(block), c);
         return cudaGetLastError();
     }
     const cudaError_t e = ensure_smem(quant_weights_kernel<SET, false>, smem);
     if (e != cudaSuccess) return e;
     quant_weights_kernel<SET, false><<<(unsigned)grid, threads, smem, s>>>(w, n_out, n_in, R, G, lo, hi, codes,
-                                                                           scales, row_mse, 0, 1.0f);
+                                                                           scales, zeros, row_mse, 0, 1.0f);
     return cudaGetLastError();
 }
 
@@ -314,12 +359,19 @@ cudaError_t launch_quantize_weights(const float* w, int64_t n_out, int64_t n_in,
                                     int block) {
     if (n_out == 0) return cudaSuccess;
     switch (set) {
-        case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
-        case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
-        case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
-        case kSetInt4: return launch_qw<kSetInt4>(w, n_out, n_in, G, lo, hi, codes, scales, row_mse, block, s);
+        case kSetQift: return launch_qw<kSetQift>(w, n_out, n_in, G, lo, hi, codes, scales, nullptr, row_mse, block, s);
+        case kSetPot: return launch_qw<kSetPot>(w, n_out, n_in, G, lo, hi, codes, scales, nullptr, row_mse, block, s);
+        case kSetStd: return launch_qw<kSetStd>(w, n_out, n_in, G, lo, hi, codes, scales, nullptr, row_mse, block, s);
+        case kSetInt4: return launch_qw<kSetInt4>(w, n_out, n_in, G, lo, hi, codes, scales, nullptr, row_mse, block, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_quantize_weights_asym(const float* w, int64_t n_out, int64_t n_in, int G, double lo, double hi,
+                                         uint32_t* codes, float* scales, int32_t* zeros, double* row_mse,
+                                         cudaStream_t s) {
+    if (n_out == 0) return cudaSuccess;
+    return launch_qw<kSetAsym>(w, n_out, n_in, G, lo, hi, codes, scales, zeros, row_mse, 0, s);
 }
 
 }  // namespace qift
