@@ -75,9 +75,13 @@ def qift_status_string(status: int) -> str:
     return lib().qift_status_string(int(status)).decode()
 
 
-def _stream(stream):
+def _stream(stream, device=None):
+    """The stream to launch on: `stream`, else the current stream of `device` (the device the
+    call's tensors live on)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
     return C.c_void_p(stream.cuda_stream)
 
 
@@ -92,6 +96,37 @@ def _cuda(t: torch.Tensor, name: str, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _same_device(*named):
+    """All given (name, tensor) pairs (None tensors skipped) on one CUDA device; returns it."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if dev is None:
+            dev, first = t.device, name
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, {first} on {dev}: every tensor of a call must be on one device")
+    return dev
+
+
+def _shape(t: torch.Tensor, name: str, shape: tuple):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _at_least(t: torch.Tensor, name: str, n: int):
+    if t.numel() < n:
+        raise ValueError(f"{name} must hold at least {n} elements, got {t.numel()}")
+    return t
+
+
+def _2d(t: torch.Tensor, name: str):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
     return t
 
 
@@ -114,11 +149,17 @@ def qift_rotate(x: torch.Tensor, block: int, out: torch.Tensor | None = None, st
     _cuda(x, "x")
     if x.dtype not in (torch.float32, torch.float16):
         raise ValueError("x must be float32 or float16")
-    y = torch.empty_like(x) if out is None else _cuda(out, "out", x.dtype)
+    if x.dim() == 0:
+        raise ValueError("x must have at least one dimension")
+    if out is not None:
+        _shape(_cuda(out, "out", x.dtype), "out", x.shape)
+    dev = _same_device(("x", x), ("out", out))
+    y = torch.empty_like(x) if out is None else out
     n = x.shape[-1]
     rows = x.numel() // n if n else 0
     dt = QIFT_F32 if x.dtype == torch.float32 else QIFT_F16
-    _check(lib().qift_rotate(_ptr(x), _ptr(y), dt, rows, n, block, _stream(stream)), "qift_rotate")
+    with torch.cuda.device(dev):
+        _check(lib().qift_rotate(_ptr(x), _ptr(y), dt, rows, n, block, _stream(stream, dev)), "qift_rotate")
     return y
 
 
@@ -129,15 +170,16 @@ def qift_quantize_weights(w_rot: torch.Tensor, levelset="qift", grid_points: int
     Returns ``(codes int32-viewed-as-u32 [N, K/16] ([N, K/8] for "int4"), scales f32 [N],
     row_mse f64 [N] or None)``.
     """
-    _cuda(w_rot, "w_rot", torch.float32)
+    _2d(_cuda(w_rot, "w_rot", torch.float32), "w_rot")
     n_out, n_in = w_rot.shape
     dev = w_rot.device
     codes = torch.empty((n_out, n_in // _codes_per_word(levelset)), dtype=torch.int32, device=dev)
     scales = torch.empty(n_out, dtype=torch.float32, device=dev)
     mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
-    _check(lib().qift_quantize_weights(_ptr(w_rot), n_out, n_in, _set(levelset), grid_points, lo, hi,
-                                       _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
-           "qift_quantize_weights")
+    with torch.cuda.device(dev):
+        _check(lib().qift_quantize_weights(_ptr(w_rot), n_out, n_in, _set(levelset), grid_points, lo, hi,
+                                           _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream, dev)),
+               "qift_quantize_weights")
     return codes, scales, mse
 
 
@@ -148,16 +190,17 @@ def qift_quantize_weights_asym(w_rot: torch.Tensor, grid_points: int = 100, lo: 
     Returns ``(codes int32-viewed-as-u32 [N, K/16], scales f32 [N], zeros int32 [N],
     row_mse f64 [N] or None)``.
     """
-    _cuda(w_rot, "w_rot", torch.float32)
+    _2d(_cuda(w_rot, "w_rot", torch.float32), "w_rot")
     n_out, n_in = w_rot.shape
     dev = w_rot.device
     codes = torch.empty((n_out, n_in // 16), dtype=torch.int32, device=dev)
     scales = torch.empty(n_out, dtype=torch.float32, device=dev)
     zeros = torch.empty(n_out, dtype=torch.int32, device=dev)
     mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
-    _check(lib().qift_quantize_weights_asym(_ptr(w_rot), n_out, n_in, grid_points, lo, hi, _ptr(codes),
-                                            _ptr(scales), _ptr(zeros), _ptr(mse), _stream(stream)),
-           "qift_quantize_weights_asym")
+    with torch.cuda.device(dev):
+        _check(lib().qift_quantize_weights_asym(_ptr(w_rot), n_out, n_in, grid_points, lo, hi, _ptr(codes),
+                                                _ptr(scales), _ptr(zeros), _ptr(mse), _stream(stream, dev)),
+               "qift_quantize_weights_asym")
     return codes, scales, zeros, mse
 
 
@@ -165,50 +208,62 @@ def qift_rotate_quantize_weights(w: torch.Tensor, block: int, levelset="qift", g
                                  lo: float = 0.2, hi: float = 1.0, with_mse: bool = True, stream=None):
     """Rotation (block b; 0 = none) + scale search + encode + pack in one pass over the raw
     weights.  Same outputs, bit for bit, as ``qift_quantize_weights(qift_rotate(w, b))``."""
-    _cuda(w, "w", torch.float32)
+    _2d(_cuda(w, "w", torch.float32), "w")
     n_out, n_in = w.shape
     dev = w.device
     codes = torch.empty((n_out, n_in // _codes_per_word(levelset)), dtype=torch.int32, device=dev)
     scales = torch.empty(n_out, dtype=torch.float32, device=dev)
     mse = torch.empty(n_out, dtype=torch.float64, device=dev) if with_mse else None
-    _check(lib().qift_rotate_quantize_weights(_ptr(w), n_out, n_in, block, _set(levelset), grid_points, lo, hi,
-                                              _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream)),
-           "qift_rotate_quantize_weights")
+    with torch.cuda.device(dev):
+        _check(lib().qift_rotate_quantize_weights(_ptr(w), n_out, n_in, block, _set(levelset), grid_points, lo,
+                                                  hi, _ptr(codes), _ptr(scales), _ptr(mse), _stream(stream, dev)),
+               "qift_rotate_quantize_weights")
     return codes, scales, mse
 
 
 def qift_quantize_acts(x: torch.Tensor, block: int = 0, out_q: torch.Tensor | None = None,
                        out_scales: torch.Tensor | None = None, stream=None):
     """Optional rotation + symmetric per-token INT4.  Returns ``(q int8 [T, K], s_a f32 [T])``."""
-    _cuda(x, "x", torch.float16)
+    _2d(_cuda(x, "x", torch.float16), "x")
     T, K = x.shape
-    q = torch.empty((T, K), dtype=torch.int8, device=x.device) if out_q is None else _cuda(out_q, "out_q", torch.int8)
-    s = torch.empty(T, dtype=torch.float32, device=x.device) if out_scales is None else \
-        _cuda(out_scales, "out_scales", torch.float32)
-    _check(lib().qift_quantize_acts(_ptr(x), T, K, block, _ptr(q), _ptr(s), _stream(stream)), "qift_quantize_acts")
+    if out_q is not None:
+        _shape(_cuda(out_q, "out_q", torch.int8), "out_q", (T, K))
+    if out_scales is not None:
+        _at_least(_cuda(out_scales, "out_scales", torch.float32), "out_scales", T)
+    dev = _same_device(("x", x), ("out_q", out_q), ("out_scales", out_scales))
+    q = torch.empty((T, K), dtype=torch.int8, device=dev) if out_q is None else out_q
+    s = torch.empty(T, dtype=torch.float32, device=dev) if out_scales is None else out_scales
+    with torch.cuda.device(dev):
+        _check(lib().qift_quantize_acts(_ptr(x), T, K, block, _ptr(q), _ptr(s), _stream(stream, dev)),
+               "qift_quantize_acts")
     return q, s
 
 
 def qift_quantize_kv(x: torch.Tensor, block: int, stream=None):
     """KV4: rotation by ``block`` + per-token INT4, two codes per byte.
     Returns ``(packed uint8 [T, n/2], scales f32 [T])``."""
-    _cuda(x, "x", torch.float16)
+    _2d(_cuda(x, "x", torch.float16), "x")
     T, n = x.shape
-    packed = torch.empty((T, n // 2), dtype=torch.uint8, device=x.device)
-    scales = torch.empty(T, dtype=torch.float32, device=x.device)
-    _check(lib().qift_quantize_kv(_ptr(x), T, n, block, _ptr(packed), _ptr(scales), _stream(stream)),
-           "qift_quantize_kv")
+    dev = x.device
+    packed = torch.empty((T, n // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(T, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().qift_quantize_kv(_ptr(x), T, n, block, _ptr(packed), _ptr(scales), _stream(stream, dev)),
+               "qift_quantize_kv")
     return packed, scales
 
 
 def qift_dequantize_kv(packed: torch.Tensor, scales: torch.Tensor, block: int, stream=None) -> torch.Tensor:
     """Inverse of ``qift_quantize_kv`` up to the quantization error: fp16 [T, n]."""
-    _cuda(packed, "packed", torch.uint8)
+    _2d(_cuda(packed, "packed", torch.uint8), "packed")
     _cuda(scales, "scales", torch.float32)
     T, n2 = packed.shape
-    out = torch.empty((T, 2 * n2), dtype=torch.float16, device=packed.device)
-    _check(lib().qift_dequantize_kv(_ptr(packed), _ptr(scales), T, 2 * n2, block, _ptr(out), _stream(stream)),
-           "qift_dequantize_kv")
+    _at_least(scales, "scales", T)
+    dev = _same_device(("packed", packed), ("scales", scales))
+    out = torch.empty((T, 2 * n2), dtype=torch.float16, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().qift_dequantize_kv(_ptr(packed), _ptr(scales), T, 2 * n2, block, _ptr(out),
+                                        _stream(stream, dev)), "qift_dequantize_kv")
     return out
 
 
@@ -222,15 +277,25 @@ def qift_linear(q: torch.Tensor, act_scale: torch.Tensor, codes: torch.Tensor, w
     _cuda(w_scale, "w_scale", torch.float32)
     if codes.dtype not in (torch.int32, torch.uint32):
         raise ValueError("codes must be 32-bit words")
+    if out_dtype not in (torch.float16, torch.float32):
+        raise ValueError("out_dtype must be torch.float16 or torch.float32")
+    _2d(q, "q")
+    _2d(codes, "codes")
     T, K = q.shape
     N = codes.shape[0]
     cpw = _codes_per_word(levelset)
     if codes.shape[1] * cpw != K:
         raise ValueError(f"codes must be [n_out, n_in/{cpw}]")
-    y = torch.empty((T, N), dtype=out_dtype, device=q.device) if out is None else _cuda(out, "out", out_dtype)
+    _at_least(act_scale, "act_scale", T)
+    _at_least(w_scale, "w_scale", N)
+    if out is not None:
+        _shape(_cuda(out, "out", out_dtype), "out", (T, N))
+    dev = _same_device(("q", q), ("act_scale", act_scale), ("codes", codes), ("w_scale", w_scale), ("out", out))
+    y = torch.empty((T, N), dtype=out_dtype, device=dev) if out is None else out
     dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
-    _check(lib().qift_linear(_ptr(q), _ptr(act_scale), _ptr(codes), _ptr(w_scale), _set(levelset), T, N, K,
-                             _ptr(y), dt, _stream(stream)), "qift_linear")
+    with torch.cuda.device(dev):
+        _check(lib().qift_linear(_ptr(q), _ptr(act_scale), _ptr(codes), _ptr(w_scale), _set(levelset), T, N, K,
+                                 _ptr(y), dt, _stream(stream, dev)), "qift_linear")
     return y
 
 
@@ -241,19 +306,32 @@ def qift_decode_linear(x: torch.Tensor, block: int, codes: torch.Tensor, w_scale
     _cuda(x, "x", torch.float16)
     _cuda(codes, "codes")
     _cuda(w_scale, "w_scale", torch.float32)
+    if codes.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("codes must be 32-bit words")
+    if out_dtype not in (torch.float16, torch.float32):
+        raise ValueError("out_dtype must be torch.float16 or torch.float32")
+    _2d(x, "x")
+    _2d(codes, "codes")
     T, K = x.shape
     N = codes.shape[0]
     cpw = _codes_per_word(levelset)
     if codes.shape[1] * cpw != K:
         raise ValueError(f"codes must be [n_out, n_in/{cpw}]")
-    y = torch.empty((T, N), dtype=out_dtype, device=x.device) if out is None else _cuda(out, "out", out_dtype)
+    _at_least(w_scale, "w_scale", N)
+    if out is not None:
+        _shape(_cuda(out, "out", out_dtype), "out", (T, N))
     if q_out is not None:
-        _cuda(q_out, "q_out", torch.int8)
+        _shape(_cuda(q_out, "q_out", torch.int8), "q_out", (T, K))
     if act_scale_out is not None:
-        _cuda(act_scale_out, "act_scale_out", torch.float32)
+        _at_least(_cuda(act_scale_out, "act_scale_out", torch.float32), "act_scale_out", T)
+    dev = _same_device(("x", x), ("codes", codes), ("w_scale", w_scale), ("out", out), ("q_out", q_out),
+                       ("act_scale_out", act_scale_out))
+    y = torch.empty((T, N), dtype=out_dtype, device=dev) if out is None else out
     dt = QIFT_F16 if out_dtype == torch.float16 else QIFT_F32
-    _check(lib().qift_decode_linear(_ptr(x), T, K, block, _ptr(codes), _ptr(w_scale), _set(levelset), N, _ptr(y), dt,
-                                    _ptr(q_out), _ptr(act_scale_out), _stream(stream)), "qift_decode_linear")
+    with torch.cuda.device(dev):
+        _check(lib().qift_decode_linear(_ptr(x), T, K, block, _ptr(codes), _ptr(w_scale), _set(levelset), N, _ptr(y),
+                                        dt, _ptr(q_out), _ptr(act_scale_out), _stream(stream, dev)),
+               "qift_decode_linear")
     return y
 
 
