@@ -165,14 +165,16 @@ qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64
  *   q_act     : int8 [tokens][n_in] from qift_quantize_acts.  act_scale: fp32 [tokens].
  *   codes     : u32 [n_out][n_in/16], w_scale: fp32 [n_out], from qift_quantize_weights.
  *   set       : QIFT_SET_QIFT or QIFT_SET_POT (QIFT_SET_STD -> QIFT_ERR_UNSUPPORTED), or
- *               QIFT_SET_INT4 (W4A4: codes u32 [n_out][n_in/8]; 1..16 tokens and n_in % 64 == 0,
- *               else QIFT_ERR_UNSUPPORTED; acc = sum q * level, |acc| <= 8*7*n_in; one token
- *               on CUDA cores, 2..16 on the int8 tensor cores).
+ *               QIFT_SET_INT4 (W4A4: codes u32 [n_out][n_in/8]; n_in % 64 == 0, else
+ *               QIFT_ERR_UNSUPPORTED; acc = sum q * level, |acc| <= 7*7*n_in; one token on CUDA
+ *               cores, 2..16 on the int8 tensor cores (mma.sync), 17 or more on the tcgen05 GEMM).
  *   y         : [tokens][n_out] out, out_dt QIFT_F32 or QIFT_F16 (round to nearest even).
  *   n_in      : multiple of 16, at most 32768 (so |acc| <= 7*4*n_in < 2^24 and (float)acc is
  *               exact).  tokens == 0 or n_out == 0 is a no-op.
  * Decode-size batches (tokens <= 16) run as an HBM-streaming GEMV; larger batches as an int8
- * tensor-core GEMM (n_in % 64 == 0; otherwise the GEMV).  Both give bit-identical results.
+ * tensor-core GEMM, which needs n_in % 64 == 0: tokens >= 17 with another n_in returns
+ * QIFT_ERR_UNSUPPORTED (pad n_in to a multiple of 64 with zero activations -- any code in the
+ * padded positions then contributes nothing).  All paths give bit-identical results.
  * Overlap: the decode kernels are launched as programmatic dependents of the previous kernel
  * on `stream` and may start reading the weights -- `codes` and `w_scale`, nothing else --
  * before that kernel has finished; the values of q_act and act_scale are read, and y written,
@@ -207,7 +209,10 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
 
 /* qift_device_error -- synchronise `stream`, then read and clear the device error word.
  * Returns QIFT_OK, QIFT_ERR_TIMEOUT (a bounded on-chip wait gave up; that call's output is
- * invalid) or QIFT_ERR_CUDA.  *detail (may be NULL) receives the raw word. */
+ * invalid) or QIFT_ERR_CUDA.  *detail (may be NULL) receives the raw word.  The word is one per
+ * device (the current one), not per stream or per call: a timeout of a kernel on any stream of
+ * the device is reported to -- and cleared by -- whichever caller reads it first, so a caller
+ * that runs work on several streams should synchronise them before reading it. */
 qift_status qift_device_error(void* stream, int32_t* detail);
 
 /* Human-readable name of a status.  Never NULL. */

@@ -16,35 +16,36 @@ extern "C" {
 
 /* Give every on-chip wait of later tensor-core GEMM and one-token launches at most `cycles` SM
  * clock cycles before it gives up (default about 4e9, some two seconds).  cycles <= 0 restores
- * the default.  Process-wide; not thread-safe against concurrent qift_linear calls. */
+ * the default.  Per host thread: it applies to the launches that thread makes. */
 qift_status qift_debug_set_wait_limit(int64_t cycles);
 
 /* Make the next tensor-core GEMM launch (qift_linear with tokens >= 17) wait, in its MMA-issuing
  * thread, on a barrier that nothing ever arrives on.  That wait runs out after the wait limit,
  * the kernel abandons its tile, drains its copies, frees tensor memory and exits; the output is
- * left unspecified and qift_device_error() then reports QIFT_ERR_TIMEOUT.  One-shot. */
+ * left unspecified and qift_device_error() then reports QIFT_ERR_TIMEOUT.  One-shot, per host
+ * thread. */
 qift_status qift_debug_stall_next_gemm(void);
 
 /* Make the next one-token launch (qift_linear or qift_decode_linear with tokens == 1) wait for
  * its staged codes on a barrier that nothing ever arrives on.  That wait runs out after the
  * wait limit; every CTA then waits for its own copies to land and exits without writing its
- * outputs, and qift_device_error() reports QIFT_ERR_TIMEOUT.  One-shot. */
+ * outputs, and qift_device_error() reports QIFT_ERR_TIMEOUT.  One-shot, per host thread. */
 qift_status qift_debug_stall_next_one_token(void);
 
 /* Turn programmatic dependent launch of the decode-size kernels on (default) or off, to
- * measure what the overlap with the previous kernel is worth.  Process-wide. */
+ * measure what the overlap with the previous kernel is worth.  Per host thread. */
 qift_status qift_debug_set_pdl(int32_t enable);
 
 /* Pin the kernel family qift_linear uses: 0 = automatic (by batch size), 1 = CUDA-core GEMV
- * (warps stream their rows' codes into registers), 2 = tensor-core skinny GEMM (tokens <= 16,
- * n_in % 64 == 0), 3 = tcgen05 GEMM with the decoded weights in shared memory, 4 = tcgen05 GEMM
- * with the decoded weights in tensor memory, 5 = its persistent form with two accumulators,
- * 6 = its CTA-pair form (two SMs per tile, tcgen05 cta_group::2), 7 = the one-token kernel
- * (tokens == 1, codes bulk-copied into shared memory); 3 to 7 need n_in % 64 == 0.  A pinned
- * family that cannot take a call makes it return QIFT_ERR_UNSUPPORTED.  qift_decode_linear with
- * one token uses the one-token kernel under 0 and 7 and its warp-per-row kernel under any other
- * pin.  All families give bit-identical results; tests use this to cover each on the same
- * inputs.  Process-wide. */
+ * (warps stream their rows' codes into registers; at most 4 * 65535 tokens), 2 = tensor-core
+ * skinny GEMM (tokens <= 16, n_in % 64 == 0), 6 = the tcgen05 GEMM on CTA pairs (two SMs per
+ * tile, cta_group::2, decoded weights in tensor memory; n_in % 64 == 0), 7 = the one-token kernel
+ * (tokens == 1, codes bulk-copied into shared memory).  Other values return
+ * QIFT_ERR_INVALID_ARG.  A pinned family that cannot take a call makes it return
+ * QIFT_ERR_UNSUPPORTED.  qift_decode_linear with one token uses the one-token kernel under 0 and
+ * 7 and its warp-per-row kernel under any other pin.  All families give bit-identical results;
+ * tests use this to cover each on the same inputs.  The pin is per host thread: it changes
+ * only the calls that thread makes. */
 qift_status qift_debug_set_linear_path(int32_t path);
 
 #ifdef __cplusplus

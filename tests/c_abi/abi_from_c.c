@@ -47,8 +47,10 @@ int main(void) {
 
     expect("linear: standard set", qift_linear(fake, fake, fake, fake, QIFT_SET_STD, 1, 8, 64, fake, QIFT_F16, NULL),
            QIFT_ERR_UNSUPPORTED);
-    expect("linear: 4-bit, 17 tokens",
-           qift_linear(fake, fake, fake, fake, QIFT_SET_INT4, 17, 8, 64, fake, QIFT_F16, NULL), QIFT_ERR_UNSUPPORTED);
+    expect("linear: 17 tokens, n_in not a multiple of 64",
+           qift_linear(fake, fake, fake, fake, QIFT_SET_QIFT, 17, 8, 80, fake, QIFT_F16, NULL), QIFT_ERR_UNSUPPORTED);
+    expect("linear: 4-bit, n_in not a multiple of 64",
+           qift_linear(fake, fake, fake, fake, QIFT_SET_INT4, 17, 8, 48, fake, QIFT_F16, NULL), QIFT_ERR_UNSUPPORTED);
     expect("linear: no tokens", qift_linear(NULL, NULL, NULL, NULL, QIFT_SET_QIFT, 0, 8, 64, NULL, QIFT_F32, NULL),
            QIFT_OK);
 

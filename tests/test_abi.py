@@ -115,9 +115,13 @@ def test_linear_validation(L):
     assert f(FAKE, FAKE, FAKE, FAKE, 0, 1, 8, 65536, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
     assert f(None, None, None, None, 0, 0, 8, 64, None, 1, None) == q.QIFT_OK                # no tokens
     assert f(None, None, None, None, 1, 3, 0, 64, None, 0, None) == q.QIFT_OK                # no outputs
-    # 4-bit weights (set 3): 1..16 tokens, n_in a multiple of 64; zero tokens is still a no-op
+    # prefill sizes (>= 17 tokens) need n_in % 64 == 0 for the tensor cores: refused, not run on
+    # the CUDA-core GEMV
+    assert f(FAKE, FAKE, FAKE, FAKE, 0, 17, 8, 80, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 1, 2048, 8, 4112, FAKE, 0, None) == q.QIFT_ERR_UNSUPPORTED
+    # 4-bit weights (set 3): any batch, n_in a multiple of 64; zero tokens is still a no-op
     assert f(FAKE, FAKE, FAKE, FAKE, 4, 1, 8, 64, FAKE, 1, None) == bad                      # set
-    assert f(FAKE, FAKE, FAKE, FAKE, 3, 17, 8, 64, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, 3, 17, 8, 48, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
     assert f(FAKE, FAKE, FAKE, FAKE, 3, 2, 8, 48, FAKE, 1, None) == q.QIFT_ERR_UNSUPPORTED
     assert f(None, None, None, None, 3, 0, 8, 64, None, 1, None) == q.QIFT_OK
 

@@ -281,7 +281,7 @@ def test_linear_w4_extreme_accumulators():
     s_a = np.ones(T, np.float32)
     y, acc = oracle.linear_w4(q, s_a, codes, s_w, np.float32)
     assert np.abs(acc).max() == 49 * K
-    for pin in ("skinny", "gemv"):
+    for pin in ("skinny", "gemv", "gemm_pair"):
         qg.qift_debug_set_linear_path(pin)
         try:
             gy = qg.qift_linear(dev(q), dev(s_a), dev(codes.view(np.int32)), dev(s_w), "int4", torch.float32)
@@ -290,20 +290,38 @@ def test_linear_w4_extreme_accumulators():
         assert np.array_equal(host(gy), y), pin
 
 
+@pytest.mark.parametrize("pin", ["auto", "gemm_pair"])
+@pytest.mark.parametrize("T,N,K", [(17, 256, 64), (128, 256, 128), (129, 257, 192), (300, 600, 4096), (256, 40, 640),
+                                   (2048, 512, 11008), (64, 1000, 4160), (513, 130, 1024), (33, 64, 32768)])
+def test_linear_w4_gemm_parity(pin, T, N, K):
+    # 4-bit weights at prefill sizes on the tcgen05 pair GEMM: ragged token and row tiles, K not a
+    # multiple of the 128-input ring stage (4160, 192), the largest n_in.
+    qg.qift_debug_set_linear_path(pin)
+    try:
+        for out_dtype in (torch.float32, torch.float16):
+            got, ref = _linear_w4_case(T, N, K, 7 * T + N + K, out_dtype)
+            u = np.uint16 if out_dtype == torch.float16 else np.uint32
+            assert np.array_equal(got.view(u), ref.view(u)), (pin, T, N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
 def test_linear_w4_unsupported_shapes_and_decode():
     rng = np.random.default_rng(1)
     K, N = 128, 16
     codes = dev(rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32).view(np.int32))
     s_w = dev(np.ones(N, np.float32))
-    for T in (17, 64):                                         # more tokens than the 4-bit kernel takes
-        q = dev(np.zeros((T, K), np.int8))
-        with pytest.raises(qg.QiftError):
-            qg.qift_linear(q, dev(np.ones(T, np.float32)), codes, s_w, "int4", torch.float32)
     q48 = dev(np.zeros((2, 48), np.int8))                      # n_in not a multiple of 64
     with pytest.raises(qg.QiftError):
         qg.qift_linear(q48, dev(np.ones(2, np.float32)), dev(np.zeros((N, 6), np.int32)), s_w, "int4")
-    with pytest.raises(qg.QiftError):                          # no one-launch decode for 4-bit weights
-        qg.qift_decode_linear(dev(np.zeros((1, K), np.float16)), 128, codes, s_w, "int4")
+    q20 = dev(np.zeros((20, K), np.int8))                      # the CUDA-core GEMV takes at most 16 tokens
+    qg.qift_debug_set_linear_path("gemv")
+    try:
+        with pytest.raises(qg.QiftError):
+            qg.qift_linear(q20, dev(np.ones(20, np.float32)), codes, s_w, "int4")
+    finally:
+        qg.qift_debug_set_linear_path("auto")
     y = qg.qift_linear(dev(np.zeros((0, K), np.int8)), dev(np.ones(0, np.float32)), codes, s_w, "int4")
     assert y.shape == (0, N)
 
@@ -493,7 +511,7 @@ def test_linear_one_token_extreme_accumulators():
 
 
 # ------------------------------------------------------------- tensor-core GEMM (prefill)
-@pytest.mark.parametrize("path", ["gemm", "gemm_ts", "gemm_tsp", "gemm_pair"])
+@pytest.mark.parametrize("path", ["auto", "gemm_pair"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(17, 256, 64), (128, 256, 128), (129, 257, 192), (300, 600, 4096),
                                     (256, 40, 640), (2048, 512, 11008), (64, 1000, 4160), (513, 130, 1024)])
@@ -511,7 +529,7 @@ def test_linear_gemm_parity(path, name, T, N, K):
 
 
 # ------------------------------------------------------- every kernel family, same inputs
-@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm", "gemm_ts", "gemm_tsp", "gemm_pair"])
+@pytest.mark.parametrize("path", ["gemv", "skinny", "gemm_pair"])
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("T,N,K", [(1, 300, 4096), (2, 129, 512), (7, 64, 1024), (9, 257, 14336), (16, 4096, 4096),
                                     (16, 130, 64), (5, 1000, 11008)])
@@ -525,6 +543,35 @@ def test_linear_each_kernel_family(path, name, T, N, K):
     finally:
         qg.qift_debug_set_linear_path("auto")
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
+def test_prefill_with_unaligned_inputs_is_refused_not_slow():
+    """Seventeen or more tokens run on the tensor cores only; an n_in they cannot take (not a
+    multiple of 64) is refused, not sent to the CUDA-core GEMV.  Pinned to the GEMV the same call
+    still runs, and matches the oracle."""
+    T, N, K = 64, 96, 4112
+    q = torch.zeros((T, K), dtype=torch.int8, device="cuda")
+    codes = torch.zeros((N, K // 16), dtype=torch.int32, device="cuda")
+    with pytest.raises(qg.QiftError) as e:
+        qg.qift_linear(q, torch.ones(T, device="cuda"), codes, torch.ones(N, device="cuda"), "qift")
+    assert e.value.status == qg.QIFT_ERR_UNSUPPORTED
+    qg.qift_debug_set_linear_path("gemv")
+    try:
+        got, ref = _linear_case("qift", T, N, K, 4112, torch.float32)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # 16 tokens with the same n_in stay on the decode-size GEMV
+    got, ref = _linear_case("pot", 16, N, K, 4113, torch.float16)
+    assert np.array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
+def test_removed_gemm_pins_are_invalid():
+    for p in (3, 4, 5, 8, -1):
+        with pytest.raises(qg.QiftError) as e:
+            qg.qift_debug_set_linear_path(p)
+        assert e.value.status == qg.QIFT_ERR_INVALID_ARG
+    qg.qift_debug_set_linear_path("auto")
 
 
 def test_pinned_family_rejects_unsupported_shape():

@@ -358,12 +358,12 @@ def qift_debug_stall_next_one_token() -> None:
     _check(lib().qift_debug_stall_next_one_token(), "qift_debug_stall_next_one_token")
 
 
-LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm": 3, "gemm_ts": 4, "gemm_tsp": 5, "gemm_pair": 6,
-                "one_token": 7}
+LINEAR_PATHS = {"auto": 0, "gemv": 1, "skinny": 2, "gemm_pair": 6, "one_token": 7}
 
 
 def qift_debug_set_linear_path(path) -> None:
-    """Test hook: pin qift_linear's kernel family ("auto", "gemv", "skinny", "gemm")."""
+    """Test hook: pin qift_linear's kernel family in this thread ("auto", "gemv", "skinny",
+    "gemm_pair", "one_token")."""
     p = LINEAR_PATHS[path] if isinstance(path, str) else int(path)
     _check(lib().qift_debug_set_linear_path(p), "qift_debug_set_linear_path")
 

@@ -27,8 +27,10 @@ bool valid_block(int64_t b) { return is_pow2(b) && b >= 2 && b <= 4096; }
 
 namespace qift {
 
-static int g_linear_path = kPathAuto;
-static bool g_pdl = true;
+// Debug pins (qift_debug.h), per host thread, so a pin set by one thread never changes the
+// kernels another thread's calls launch.
+static thread_local int g_linear_path = kPathAuto;
+static thread_local bool g_pdl = true;
 void debug_set_pdl(bool on) { g_pdl = on; }
 bool pdl_enabled() { return g_pdl; }
 void debug_set_linear_path(int path) { g_linear_path = path; }
@@ -176,29 +178,42 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
     const bool f16 = out_dt == QIFT_F16;
     int path = qift::debug_linear_path();
     if (set == QIFT_SET_INT4) {
-        // 4-bit weights: the tensor-core skinny kernel for 2..16 tokens, the CUDA-core GEMV for one
-        // token; pinning "skinny" forces the former, any other pin the latter.
-        if (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in))
-            return QIFT_ERR_UNSUPPORTED;
-        const bool skinny = path == qift::kPathSkinny ||
-                            (path == qift::kPathAuto && tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in));
-        if (skinny)
+        // 4-bit weights: the tcgen05 pair GEMM from 17 tokens, the tensor-core skinny kernel for
+        // 2..16, the CUDA-core GEMV for one; pinning "gemm_pair" or "skinny" forces that family,
+        // any other pin the GEMV (which takes at most 16 tokens).
+        if (path == qift::kPathAuto)
+            path = tokens >= qift::kGemmMinTokens
+                       ? qift::kPathGemmPair
+                       : (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in) ? qift::kPathSkinny
+                                                                                            : qift::kPathGemv);
+        if (path == qift::kPathGemmPair) {
+            if (!qift::linear_gemm_supported(tokens, n_out, n_in)) return QIFT_ERR_UNSUPPORTED;
+            return from_cuda(qift::launch_linear_gemm_pair(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
+                                                           n_in, y, f16, s));
+        }
+        if (path == qift::kPathSkinny) {
+            if (!qift::linear_skinny_supported(tokens, n_out, n_in)) return QIFT_ERR_UNSUPPORTED;
             return from_cuda(qift::launch_linear_skinny(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
                                                         n_in, y, f16, s));
+        }
+        if (tokens > 16) return QIFT_ERR_UNSUPPORTED;
         return from_cuda(qift::launch_linear_w4(q_act, act_scale, codes, w_scale, tokens, n_out, n_in, y, f16, s));
     }
     if (path == qift::kPathAuto) {
-        if (tokens >= qift::kGemmMinTokens && qift::linear_gemm_supported(tokens, n_out, n_in))
+        if (tokens >= qift::kGemmMinTokens) {
+            // Prefill sizes run on the tensor cores only.  The code matrix's rows must be 16-byte
+            // multiples for the tensor-memory copies (n_in % 64 == 0); any other n_in is refused
+            // rather than sent to the CUDA-core GEMV, whose cost grows with every token.
+            if (!qift::linear_gemm_supported(tokens, n_out, n_in)) return QIFT_ERR_UNSUPPORTED;
             path = qift::kPathGemmPair;
-        else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
+        } else if (tokens >= 2 && qift::linear_skinny_supported(tokens, n_out, n_in))
             path = qift::kPathSkinny;
         else if (tokens == 1 && qift::linear_one_token_preferred(n_out, n_in))
             path = qift::kPathOneToken;
         else
             path = qift::kPathGemv;
-    } else if (((path == qift::kPathGemm || path == qift::kPathGemmTs || path == qift::kPathGemmTsp ||
-                 path == qift::kPathGemmPair) &&
-                !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
+    } else if ((path == qift::kPathGemmPair && !qift::linear_gemm_supported(tokens, n_out, n_in)) ||
+               (path == qift::kPathGemv && !qift::linear_gemv_supported(tokens)) ||
                (path == qift::kPathSkinny && !qift::linear_skinny_supported(tokens, n_out, n_in)) ||
                (path == qift::kPathOneToken && (tokens != 1 || !qift::linear_one_token_supported(n_out, n_in)))) {
         return QIFT_ERR_UNSUPPORTED;
@@ -209,15 +224,6 @@ qift_status qift_linear(const int8_t* q_act, const float* act_scale, const uint3
     if (path == qift::kPathGemmPair)
         return from_cuda(qift::launch_linear_gemm_pair(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
                                                        n_in, y, f16, s));
-    if (path == qift::kPathGemmTsp)
-        return from_cuda(qift::launch_linear_gemm_tsp(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
-                                                      n_in, y, f16, s));
-    if (path == qift::kPathGemmTs)
-        return from_cuda(qift::launch_linear_gemm_ts(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out,
-                                                     n_in, y, f16, s));
-    if (path == qift::kPathGemm)
-        return from_cuda(qift::launch_linear_gemm(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in, y,
-                                                  f16, s));
     if (path == qift::kPathSkinny)
         return from_cuda(qift::launch_linear_skinny(q_act, act_scale, codes, w_scale, (int)set, tokens, n_out, n_in,
                                                     y, f16, s));
@@ -269,7 +275,9 @@ qift_status qift_debug_set_wait_limit(int64_t cycles) {
 }
 
 qift_status qift_debug_set_linear_path(int32_t path) {
-    if (path < 0 || path > 7) return QIFT_ERR_INVALID_ARG;
+    if (path != qift::kPathAuto && path != qift::kPathGemv && path != qift::kPathSkinny &&
+        path != qift::kPathGemmPair && path != qift::kPathOneToken)
+        return QIFT_ERR_INVALID_ARG;
     qift::debug_set_linear_path(path);
     return QIFT_OK;
 }

@@ -57,7 +57,9 @@ cudaError_t launch_quantize_weights_asym(const float* w, int64_t n_out, int64_t 
                                          double hi, uint32_t* codes, float* scales, int32_t* zeros, double* row_mse,
                                          cudaStream_t s);
 
-// Decode-size linear: HBM-streaming GEMV (CUDA-core dp4a).
+// Decode-size linear: HBM-streaming GEMV (CUDA-core dp4a); its grid takes at most
+// 4 * 65535 tokens.
+bool linear_gemv_supported(int64_t tokens);
 cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
                                cudaStream_t s);
@@ -73,11 +75,11 @@ cudaError_t launch_decode_linear(const void* x, int64_t tokens, int64_t n_in, in
                                  const float* s_w, int set, int64_t n_out, void* y, bool f16, int8_t* q_out,
                                  float* sa_out, cudaStream_t s);
 
-// Prefill-size linear: tcgen05 int8 tensor-core GEMM with in-register code decode.
+// Prefill-size linear: tcgen05 int8 tensor-core GEMM on CTA pairs (cta_group::2), the decoded
+// weights as the A operand in tensor memory.
 bool linear_gemm_supported(int64_t tokens, int64_t n_out, int64_t n_in);
-cudaError_t launch_linear_gemm(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
-                               int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
-                               cudaStream_t s);
+cudaError_t launch_linear_gemm_pair(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                    int set, int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s);
 
 // One token: qift_linear, and the fused decode step, on CTAs that bulk-copy their rows'
 // codes into shared memory before waiting for the previous kernel (half an SM each).
@@ -93,19 +95,17 @@ void debug_set_one_token_wait_limit(long long cycles);
 void debug_stall_next_one_token();
 cudaError_t read_and_clear_one_token_error(int* word);
 
-// 4-bit weights (QIFT_SET_INT4), 1..16 tokens: CUDA-core W4A4 GEMV.
+// 4-bit weights (QIFT_SET_INT4): which calls the library takes, and the CUDA-core W4A4 GEMV
+// (1..16 tokens).
 bool linear_w4_supported(int64_t tokens, int64_t n_in);
 cudaError_t launch_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                              int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16, cudaStream_t s);
 
-// Test hooks behind qift_debug.h.
+// Test hooks behind qift_debug.h (numbers 3 to 5 named GEMM forms that are no longer built).
 enum LinearPath {
     kPathAuto = 0,
     kPathGemv = 1,
     kPathSkinny = 2,
-    kPathGemm = 3,
-    kPathGemmTs = 4,
-    kPathGemmTsp = 5,
     kPathGemmPair = 6,
     kPathOneToken = 7
 };
@@ -115,20 +115,6 @@ void debug_set_pdl(bool on);
 bool pdl_enabled();  // programmatic dependent launch for the decode kernels (default on)
 void debug_set_gemm_wait_limit(long long cycles);
 void debug_stall_next_gemm();
-
-// Prefill-size linear, variant with the decoded weights in tensor memory (TS MMA).
-cudaError_t launch_linear_gemm_ts(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
-                                  int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
-                                  cudaStream_t s);
-
-// Tensor-memory-A GEMM on CTA pairs (tcgen05 cta_group::2): the default prefill path.
-cudaError_t launch_linear_gemm_pair(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
-                                    int set, int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s);
-
-// Persistent tensor-memory-A GEMM (double-buffered accumulators, overlapped epilogue).
-cudaError_t launch_linear_gemm_tsp(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
-                                   int set, int64_t tokens, int64_t n_out, int64_t n_in, void* y, bool f16,
-                                   cudaStream_t s);
 
 // Synchronous read-and-clear of the device error word set by bounded on-chip waits.
 cudaError_t read_and_clear_device_error(int* word);

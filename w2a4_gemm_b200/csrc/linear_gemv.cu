@@ -269,6 +269,8 @@ static cudaError_t dispatch_gemv(const int8_t* q, const float* s_a, const uint32
     return launch_gemv_t<4, 2, 1, OutT>(q, s_a, codes, s_w, lut, T, N, K, y, s);
 }
 
+bool linear_gemv_supported(int64_t T) { return T <= (int64_t)4 * 65535; }
+
 cudaError_t launch_linear_gemv(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int set,
                                int64_t T, int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
     if (T == 0 || N == 0) return cudaSuccess;

@@ -44,8 +44,9 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz before the wai
 
 __device__ int g_error = 0;  // bit 0: a CTA's wait for its codes ran out (QIFT_ERR_TIMEOUT)
 
-static long long g_wait_limit = kWaitCycles;
-static bool g_stall_next = false;
+// Test hooks (qift_debug.h), per host thread.
+static thread_local long long g_wait_limit = kWaitCycles;
+static thread_local bool g_stall_next = false;
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* p, float v);

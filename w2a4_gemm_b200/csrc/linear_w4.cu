@@ -129,7 +129,9 @@ static cudaError_t dispatch(const int8_t* q, const float* s_a, const uint32_t* c
 
 }  // namespace w4
 
-bool linear_w4_supported(int64_t tokens, int64_t n_in) { return tokens >= 1 && tokens <= 16 && n_in % 64 == 0; }
+// Any batch: one token on this kernel, 2..16 on the skinny tensor-core kernel, more on the
+// tcgen05 pair GEMM; all need n_in % 64 == 0.
+bool linear_w4_supported(int64_t tokens, int64_t n_in) { return tokens >= 1 && n_in % 64 == 0; }
 
 cudaError_t launch_linear_w4(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, int64_t T,
                              int64_t N, int64_t K, void* y, bool f16, cudaStream_t s) {
