@@ -54,8 +54,11 @@ int main(void) {
     expect("linear: no tokens", qift_linear(NULL, NULL, NULL, NULL, QIFT_SET_QIFT, 0, 8, 64, NULL, QIFT_F32, NULL),
            QIFT_OK);
 
-    expect("decode_linear: 4-bit",
-           qift_decode_linear(fake, 1, 128, 128, fake, fake, QIFT_SET_INT4, 8, fake, QIFT_F16, NULL, NULL, NULL),
+    expect("decode_linear: five tokens",
+           qift_decode_linear(fake, 5, 128, 128, fake, fake, QIFT_SET_INT4, 8, fake, QIFT_F16, NULL, NULL, NULL),
+           QIFT_ERR_UNSUPPORTED);
+    expect("decode_linear: standard set",
+           qift_decode_linear(fake, 1, 128, 128, fake, fake, QIFT_SET_STD, 8, fake, QIFT_F16, NULL, NULL, NULL),
            QIFT_ERR_UNSUPPORTED);
     expect("quantize_kv: block", qift_quantize_kv(fake, 2, 64, 3, fake, fake, NULL), QIFT_ERR_INVALID_ARG);
     expect("dequantize_kv: no tokens", qift_dequantize_kv(NULL, NULL, 0, 64, 64, NULL, NULL), QIFT_OK);

@@ -609,6 +609,52 @@ def test_decode_linear_matches_oracle(name, T, N, K, block):
         assert np.array_equal(host(gsa).view(np.uint32), s_a.view(np.uint32))
 
 
+@pytest.mark.parametrize("pin", ["auto", "gemv"])   # gemv: one token on the warp-per-row kernel
+@pytest.mark.parametrize("T,N,K,block", [(1, 4096, 4096, 4096), (1, 37, 64, 16), (2, 300, 512, 128),
+                                          (3, 129, 11008, 128), (4, 64, 14336, 128), (1, 1, 1024, 0),
+                                          (1, 14336, 4096, 128), (1, 4096, 14336, 128), (1, 149, 16384, 2048),
+                                          (1, 28000, 4096, 128), (4, 200, 2048, 2048)])
+def test_decode_linear_w4_matches_oracle(pin, T, N, K, block):
+    # 4-bit weights through the one-launch decode: rotation + INT4 + W4A4 linear, bit-exact
+    rng = np.random.default_rng(T * 11 + N + K)
+    x = synth.activations(T, K, (T, N, K, 4), n_outliers=synth.outlier_count(K))
+    codes = rng.integers(0, 2 ** 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    s_w = rng.uniform(1e-3, 1e-2, N).astype(np.float32)
+    q, s_a, _ = oracle.quantize_acts(x, block)
+    qg.qift_debug_set_linear_path(pin)
+    try:
+        for out_dtype, npdt in ((torch.float16, np.float16), (torch.float32, np.float32)):
+            ref, _ = oracle.linear_w4(q, s_a, codes, s_w, npdt)
+            gq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+            gsa = torch.empty(T, dtype=torch.float32, device="cuda")
+            gy = qg.qift_decode_linear(dev(x), block, dev(codes.view(np.int32)), dev(s_w), "int4", out_dtype,
+                                       q_out=gq, act_scale_out=gsa)
+            u = np.uint16 if npdt == np.float16 else np.uint32
+            assert np.array_equal(host(gy).view(u), ref.view(u)), (pin, T, N, K, block)
+            assert np.array_equal(host(gq), q)
+            assert np.array_equal(host(gsa).view(np.uint32), s_a.view(np.uint32))
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
+def test_decode_linear_w4_extreme_accumulators():
+    # every activation at +7 (a token of equal entries, no rotation) against the outer levels
+    # +-7: |acc| = 49 K at the largest n_in the one-launch decode takes
+    T, N, K = 1, 8, 16384
+    x = np.full((T, K), 3.0, np.float16)
+    codes = np.full((N, K // 8), 0x77777777, np.uint32)
+    codes[1::2] = 0x99999999
+    codes[2] = 0x79797979
+    s_w = np.ones(N, np.float32)
+    q, s_a, _ = oracle.quantize_acts(x, 0)
+    assert q.min() == 7
+    ref, acc = oracle.linear_w4(q, s_a, codes, s_w, np.float32)
+    assert acc.max() == 49 * K and acc.min() == -49 * K
+    gy = qg.qift_decode_linear(dev(x), 0, dev(codes.view(np.int32)), dev(s_w), "int4", torch.float32)
+    assert np.array_equal(host(gy).view(np.uint32), ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("N,K,block", [(4096, 4096, 4096), (300, 512, 128)])
 def test_decode_linear_one_token_pinned_to_warp_per_row(name, N, K, block):

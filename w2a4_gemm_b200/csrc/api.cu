@@ -236,7 +236,6 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
                                int8_t* q_out, float* act_scale_out, void* stream) {
     if (set != QIFT_SET_QIFT && set != QIFT_SET_POT && set != QIFT_SET_STD && set != QIFT_SET_INT4)
         return QIFT_ERR_INVALID_ARG;
-    if (set == QIFT_SET_INT4) return QIFT_ERR_UNSUPPORTED;
     if (out_dt != QIFT_F32 && out_dt != QIFT_F16) return QIFT_ERR_INVALID_ARG;
     if (tokens < 0 || n_out < 0 || n_in <= 0 || n_in % 16 != 0) return QIFT_ERR_INVALID_ARG;
     if (block != 0 && (!valid_block(block) || n_in % block != 0)) return QIFT_ERR_INVALID_ARG;
@@ -248,7 +247,7 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
     if (n_out > 0x7fffffff / 2) return QIFT_ERR_UNSUPPORTED;
     const int path = qift::debug_linear_path();
     if (tokens == 1 && (path == qift::kPathAuto || path == qift::kPathOneToken) &&
-        qift::decode_one_token_supported(n_out, n_in, block))
+        qift::decode_one_token_supported(n_out, n_in, block, (int)set))
         return from_cuda(qift::launch_decode_one_token(x, n_in, block, codes, w_scale, (int)set, n_out, y,
                                                        out_dt == QIFT_F16, q_out, act_scale_out,
                                                        static_cast<cudaStream_t>(stream)));

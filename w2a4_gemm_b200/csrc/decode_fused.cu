@@ -15,6 +15,10 @@
 //      shared activations; warp reduction; fp32 epilogue.
 // The grid has one CTA per SM (or more for very tall matrices) and spreads the rows evenly,
 // so each SM streams the same share of the weights.  CTA 0 can also write q and s_a out.
+// 4-bit weights (W4, the Abstract's mixed W2/W4 layers): a word holds eight inputs as
+// two's-complement nibbles (byte j = inputs j and j + 4), so (w << 4) & 0xF0F0F0F0 and
+// w & 0xF0F0F0F0 are the int8x4 operands 16 x level of inputs 0..3 and 4..7; they meet the
+// activations in natural order, and the sum is shifted back by 4 (exact) before the epilogue.
 #include <math.h>
 
 #include <algorithm>
@@ -36,7 +40,7 @@ template <>
 __device__ __forceinline__ void store_out<__half>(__half* p, float v) { *p = __float2half_rn(v); }
 
 // TC: tokens handled (T <= TC); J: 128-word slices per K chunk.
-template <int LOGB, int TC, int J, typename OutT>
+template <int LOGB, int TC, int J, bool W4, typename OutT>
 __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __restrict__ x, int T, int64_t K, float c,
                                                              const uint32_t* __restrict__ codes,
                                                              const float* __restrict__ s_w, uint32_t lut, int64_t N,
@@ -51,7 +55,7 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
     uint8_t* qs = smem + xs_bytes + act_tbuf_bytes<LOGB>();  // TC x K int8, permuted per 16-group
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t KW = K / 16;
+    const int64_t KW = K / (W4 ? 8 : 16);  // code words per row
     const int64_t cta_r0 = (int64_t)blockIdx.x * rows_per_cta;
     const int64_t cta_r1 = min(N, cta_r0 + rows_per_cta);
     const int rpw = (rows_per_cta + WARPS - 1) / WARPS;
@@ -69,10 +73,19 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
                 const int64_t wi = base + 4 * lane + 128 * j;
                 const uint4 v = (r < nr && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
                                                          : make_uint4(0u, 0u, 0u, 0u);
-                decode_word(v.x, lut, dec[r][j][0]);
-                decode_word(v.y, lut, dec[r][j][1]);
-                decode_word(v.z, lut, dec[r][j][2]);
-                decode_word(v.w, lut, dec[r][j][3]);
+                if constexpr (W4) {
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        dec[r][j][u][0] = (w[u] << 4) & 0xF0F0F0F0u;
+                        dec[r][j][u][1] = w[u] & 0xF0F0F0F0u;
+                    }
+                } else {
+                    decode_word(v.x, lut, dec[r][j][0]);
+                    decode_word(v.y, lut, dec[r][j][1]);
+                    decode_word(v.z, lut, dec[r][j][2]);
+                    decode_word(v.w, lut, dec[r][j][3]);
+                }
             }
         }
     };
@@ -94,9 +107,13 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
             for (int64_t i = (int64_t)tid * 16; i < K; i += kActThreads * 16) {
                 const uint4 v = m == 0.0f ? make_uint4(0u, 0u, 0u, 0u) : quant16(xs + i, inv);
                 if (blockIdx.x == 0 && q_out) *reinterpret_cast<uint4*>(q_out + (int64_t)t * K + i) = v;
-                uint32_t p[4];
-                permute_acts(v, p);
-                *reinterpret_cast<uint4*>(qt + i) = make_uint4(p[0], p[1], p[2], p[3]);
+                if constexpr (W4) {
+                    *reinterpret_cast<uint4*>(qt + i) = v;  // natural order
+                } else {
+                    uint32_t p[4];
+                    permute_acts(v, p);
+                    *reinterpret_cast<uint4*>(qt + i) = make_uint4(p[0], p[1], p[2], p[3]);
+                }
             }
             if (tid == 0) {
                 sa_s[t] = m == 0.0f ? 0.0f : __fdiv_rn(m, 7.0f);
@@ -117,7 +134,32 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
     for (int r = 0; r < RMAX; ++r)
 #pragma unroll
         for (int t = 0; t < TC; ++t) acc[r][t] = 0;
-    for (int64_t base = 0; base < KW; base += 128 * J) {
+    for (int64_t base = 0; base < KW && W4; base += 128 * J) {
+        if (base > 0) load_decode(base);
+        uint2 pa[TC][J][4];  // the eight activations of each word, natural order
+#pragma unroll
+        for (int t = 0; t < TC; ++t)
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t wi = base + 4 * lane + 128 * j + u;
+                    pa[t][j][u] = wi < KW ? *reinterpret_cast<const uint2*>(qs + (int64_t)t * K + wi * 8)
+                                          : make_uint2(0u, 0u);
+                }
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            if (r >= nr) break;
+#pragma unroll
+            for (int j = 0; j < J; ++j)
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int t = 0; t < TC; ++t)
+                        acc[r][t] = dp4a(dec[r][j][u][1], pa[t][j][u].y, dp4a(dec[r][j][u][0], pa[t][j][u].x, acc[r][t]));
+        }
+    }
+    for (int64_t base = 0; base < KW && !W4; base += 128 * J) {
         if (base > 0) load_decode(base);
         uint4 pa[TC][J][4];
 #pragma unroll
@@ -157,7 +199,8 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
         if (r >= nr) break;
 #pragma unroll
         for (int t = 0; t < TC; ++t) {
-            const int sum = __reduce_add_sync(0xffffffffu, acc[r][t]);
+            int sum = __reduce_add_sync(0xffffffffu, acc[r][t]);
+            if constexpr (W4) sum >>= 4;  // exact: every product was 16 x level x q
             if (lane == ((r * TC + t) & 31) && t < T) {
                 const float v = __fmul_rn(__fmul_rn((float)sum, sw[r]), sa_s[t]);
                 store_out<OutT>(y + (int64_t)t * N + row0 + r, v);
@@ -177,7 +220,7 @@ static int sm_count() {
     return cached[dev];
 }
 
-template <int LOGB, int TC, int J, typename OutT>
+template <int LOGB, int TC, int J, bool W4, typename OutT>
 static cudaError_t launch_t(const __half* x, int64_t T, int64_t K, float c, const uint32_t* codes, const float* s_w,
                             uint32_t lut, int64_t N, OutT* y, int8_t* q_out, float* sa_out, cudaStream_t s) {
     const int64_t min_ctas = (N + WARPS * RMAX - 1) / (WARPS * RMAX);
@@ -185,7 +228,7 @@ static cudaError_t launch_t(const __half* x, int64_t T, int64_t K, float c, cons
     const int64_t rows_per_cta = (N + ctas - 1) / ctas;
     const int64_t grid = (N + rows_per_cta - 1) / rows_per_cta;
     const size_t smem = ((size_t)K * 2 + 15) / 16 * 16 + act_tbuf_bytes<LOGB>() + (size_t)TC * K;
-    cudaError_t e = ensure_smem(decode_kernel<LOGB, TC, J, OutT>, smem);
+    cudaError_t e = ensure_smem(decode_kernel<LOGB, TC, J, W4, OutT>, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -197,15 +240,19 @@ static cudaError_t launch_t(const __half* x, int64_t T, int64_t K, float c, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<LOGB, TC, J, OutT>, x, (int)T, K, c, codes, s_w, lut, N,
+    return cudaLaunchKernelEx(&cfg, decode_kernel<LOGB, TC, J, W4, OutT>, x, (int)T, K, c, codes, s_w, lut, N,
                               (int)rows_per_cta, y, q_out, sa_out);
 }
 
 template <int LOGB, typename OutT>
 static cudaError_t by_tokens(const __half* x, int64_t T, int64_t K, float c, const uint32_t* codes, const float* s_w,
                              uint32_t lut, int64_t N, OutT* y, int8_t* q_out, float* sa_out, cudaStream_t s) {
-    if (T == 1) return launch_t<LOGB, 1, 2, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
-    return launch_t<LOGB, 4, 1, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
+    if (lut == 0) {  // 4-bit weights
+        if (T == 1) return launch_t<LOGB, 1, 2, true, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
+        return launch_t<LOGB, 4, 1, true, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
+    }
+    if (T == 1) return launch_t<LOGB, 1, 2, false, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
+    return launch_t<LOGB, 4, 1, false, OutT>(x, T, K, c, codes, s_w, lut, N, y, q_out, sa_out, s);
 }
 
 template <typename OutT>
@@ -236,7 +283,7 @@ cudaError_t launch_decode_linear(const void* x, int64_t T, int64_t K, int block,
                                  const float* s_w, int set, int64_t N, void* y, bool f16, int8_t* q_out,
                                  float* sa_out, cudaStream_t s) {
     const __half* xh = static_cast<const __half*>(x);
-    const uint32_t lut = level_lut(set);
+    const uint32_t lut = set == kSetInt4 ? 0u : level_lut(set);  // 0 selects the 4-bit form
     if (f16) return fused::by_block<__half>(xh, T, K, block, codes, s_w, lut, N, static_cast<__half*>(y), q_out, sa_out, s);
     return fused::by_block<float>(xh, T, K, block, codes, s_w, lut, N, static_cast<float*>(y), q_out, sa_out, s);
 }

@@ -85,7 +85,7 @@ cudaError_t launch_linear_gemm_pair(const int8_t* q, const float* s_a, const uin
 // codes into shared memory before waiting for the previous kernel (half an SM each).
 bool linear_one_token_supported(int64_t n_out, int64_t n_in);
 bool linear_one_token_preferred(int64_t n_out, int64_t n_in);  // over the warp-per-row GEMV
-bool decode_one_token_supported(int64_t n_out, int64_t n_in, int block);
+bool decode_one_token_supported(int64_t n_out, int64_t n_in, int block, int set);
 cudaError_t launch_linear_one_token(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                     int set, int64_t n_out, int64_t n_in, void* y, bool f16, cudaStream_t s);
 cudaError_t launch_decode_one_token(const void* x, int64_t n_in, int block, const uint32_t* codes, const float* s_w,

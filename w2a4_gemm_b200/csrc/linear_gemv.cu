@@ -144,33 +144,45 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const int8_t* __r
 // registers before the kernel waits for its predecessor, so after the wait only the
 // activation token (staged once per CTA in shared memory, permuted to the decode order), the
 // dp4a products, the warp reduction and the epilogue remain on the critical path.
-template <int R, int J, typename OutT>
+// The staged token is laid out so that the warp's reads are conflict-free: word wi = base +
+// 4 l + 128 j + u (lane l, slice j, word u of the lane's 16-byte code group) sits at slot
+// base + 32 (4 j + u) + l, so each 16-byte read of a warp covers 512 contiguous bytes.  (Stored in
+// word order, lane l's reads were 64 bytes apart: a 16-way bank conflict that cost ~0.5 us per
+// launch at 4096 x 4096.)
+// ONE: the row is a single chunk (n_in <= 2048 J), so no loop over chunks is compiled.
+template <int R, int J, bool ONE, typename OutT>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv1_kernel(const int8_t* __restrict__ q,
                                                                 const float* __restrict__ s_a,
                                                                 const uint32_t* __restrict__ codes,
                                                                 const float* __restrict__ s_w, uint32_t lut,
                                                                 int64_t N, int64_t K, OutT* __restrict__ y) {
-    extern __shared__ __align__(16) uint4 acts_s[];  // K/16 permuted 16-byte groups
+    extern __shared__ __align__(16) uint4 acts_s[];  // K/16 permuted 16-byte groups (chunk-padded)
     const int lane = threadIdx.x & 31;
     const int64_t warp = (int64_t)blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
     const int64_t row0 = warp * R;
     const int64_t KW = K / 16;
 
+    // All of a chunk's code loads are issued before any of them is decoded.
+    uint4 cw[R][J];
     uint32_t dec[R][J][4][4];
     auto load_decode = [&](int64_t base) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
+        for (int r = 0; r < R; ++r)
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 const int64_t wi = base + 4 * lane + 128 * j;
-                const uint4 c = (row0 + r < N && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
-                                                              : make_uint4(0u, 0u, 0u, 0u);
-                decode_word(c.x, lut, dec[r][j][0]);
-                decode_word(c.y, lut, dec[r][j][1]);
-                decode_word(c.z, lut, dec[r][j][2]);
-                decode_word(c.w, lut, dec[r][j][3]);
+                cw[r][j] = (row0 + r < N && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
             }
-        }
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                decode_word(cw[r][j].x, lut, dec[r][j][0]);
+                decode_word(cw[r][j].y, lut, dec[r][j][1]);
+                decode_word(cw[r][j].z, lut, dec[r][j][2]);
+                decode_word(cw[r][j].w, lut, dec[r][j][3]);
+            }
     };
     load_decode(0);
     griddep_launch_dependents();
@@ -180,24 +192,25 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv1_kernel(const int8_t* __
 #pragma unroll
     for (int r = 0; r < R; ++r) sw[r] = row0 + r < N ? __ldg(s_w + row0 + r) : 0.0f;
     const float sa = __ldg(s_a);
-    for (int64_t i = threadIdx.x; i < KW; i += kGemvWarps * 32) {
+    for (int i = threadIdx.x; i < (int)KW; i += kGemvWarps * 32) {
         uint32_t p[4];
         permute_acts(__ldg(reinterpret_cast<const uint4*>(q) + i), p);
-        acts_s[i] = make_uint4(p[0], p[1], p[2], p[3]);
+        const int in = i % (128 * J);  // word within its chunk: lane (in / 4) % 32, slice in / 128
+        acts_s[i - in + 32 * (4 * (in >> 7) + (in & 3)) + ((in >> 2) & 31)] = make_uint4(p[0], p[1], p[2], p[3]);
     }
     __syncthreads();
 
     int acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0;
-    for (int64_t base = 0; base < KW; base += 128 * J) {
-        if (base > 0) load_decode(base);
+    for (int64_t base = 0; base < (ONE ? 1 : KW); base += 128 * J) {
+        if (!ONE && base > 0) load_decode(base);
 #pragma unroll
         for (int j = 0; j < J; ++j) {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int64_t wi = base + 4 * lane + 128 * j + u;
-                const uint4 a = wi < KW ? acts_s[wi] : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 a = wi < KW ? acts_s[base + 32 * (4 * j + u) + lane] : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     int v = acc[r];
@@ -218,13 +231,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv1_kernel(const int8_t* __
     }
 }
 
-template <int R, int J, typename OutT>
-static cudaError_t launch_gemv1(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+template <int R, int J, bool ONE, typename OutT>
+static cudaError_t launch_gemv1_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
                                 uint32_t lut, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
     const int64_t gx = ((N + R - 1) / R + kGemvWarps - 1) / kGemvWarps;
     if (gx > 0x7fffffff) return cudaErrorInvalidValue;
-    const size_t smem = (size_t)K;  // K/16 groups of 16 bytes
-    cudaError_t e = ensure_smem(gemv1_kernel<R, J, OutT>, smem);
+    const int64_t KW = K / 16, chunk = 128 * J;
+    const size_t smem = (size_t)((KW + chunk - 1) / chunk * chunk) * 16;  // whole chunks of 16-byte groups
+    cudaError_t e = ensure_smem(gemv1_kernel<R, J, ONE, OutT>, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)gx);
@@ -236,7 +250,14 @@ static cudaError_t launch_gemv1(const int8_t* q, const float* s_a, const uint32_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv1_kernel<R, J, OutT>, q, s_a, codes, s_w, lut, N, K, y);
+    return cudaLaunchKernelEx(&cfg, gemv1_kernel<R, J, ONE, OutT>, q, s_a, codes, s_w, lut, N, K, y);
+}
+
+template <int R, int J, typename OutT>
+static cudaError_t launch_gemv1(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
+                                uint32_t lut, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
+    if (K <= 2048 * J) return launch_gemv1_t<R, J, true, OutT>(q, s_a, codes, s_w, lut, N, K, y, s);
+    return launch_gemv1_t<R, J, false, OutT>(q, s_a, codes, s_w, lut, N, K, y, s);
 }
 
 template <int TC, int R, int J, typename OutT>

@@ -25,6 +25,10 @@
 // activations, no decode at all.  The PoT levels {-4,-1,+1,+4} are not affine in c; their codes
 // are decoded by byte permutes against the level table and meet the activations in signed dp4a.
 // Either way the int32 sum is exact, so every path gives the same bits.
+// 4-bit weights (SET = kSetInt4, the mixed W2/W4 layers): eight nibbles per word, byte j = inputs
+// j and j + 4; (w << 4) & 0xF0F0F0F0 and w & 0xF0F0F0F0 are 16 x the levels of inputs 0..3 and
+// 4..7 as signed bytes, met by the activations in natural order; the row sum is 16 x acc and is
+// shifted back (exact) in the epilogue.  A 16-byte code group then covers 32 inputs, not 64.
 #include <math.h>
 
 #include <algorithm>
@@ -72,7 +76,9 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // Qift: word m = activations 4j+m, j = 0..3 (a 4x4 byte transpose).  PoT: decode_word order.
 template <int SET>
 __device__ __forceinline__ uint4 arrange(uint4 a) {
-    if constexpr (SET == kSetQift) {
+    if constexpr (SET == kSetInt4) {
+        return a;  // natural order
+    } else if constexpr (SET == kSetQift) {
         const uint32_t t0 = prmt(a.x, a.y, 0x5140u), t1 = prmt(a.z, a.w, 0x5140u);
         const uint32_t t2 = prmt(a.x, a.y, 0x7362u), t3 = prmt(a.z, a.w, 0x7362u);
         return make_uint4(prmt(t0, t1, 0x5410u), prmt(t0, t1, 0x7632u), prmt(t2, t3, 0x5410u),
@@ -96,7 +102,18 @@ __device__ __forceinline__ int sum16(uint4 a, int s) {
 template <int SET>
 __device__ __forceinline__ int dot_group(uint4 wv, const uint4 (&a)[4]) {
     const uint32_t wd[4] = {wv.x, wv.y, wv.z, wv.w};
-    if constexpr (SET == kSetQift) {
+    if constexpr (SET == kSetInt4) {  // 32 inputs: a[0], a[1] hold their activations in order
+        constexpr uint32_t M = 0xF0F0F0F0u;
+        int s = 0;
+        s = dp4a((wd[0] << 4) & M, a[0].x, s);
+        s = dp4a(wd[0] & M, a[0].y, s);
+        s = dp4a((wd[1] << 4) & M, a[0].z, s);
+        s = dp4a(wd[1] & M, a[0].w, s);
+        s = dp4a((wd[2] << 4) & M, a[1].x, s);
+        s = dp4a(wd[2] & M, a[1].y, s);
+        s = dp4a((wd[3] << 4) & M, a[1].z, s);
+        return dp4a(wd[3] & M, a[1].w, s);
+    } else if constexpr (SET == kSetQift) {
         int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -121,15 +138,19 @@ __device__ __forceinline__ int dot_group(uint4 wv, const uint4 (&a)[4]) {
     }
 }
 
-// Shared memory after the static part: codes [R][K/64] x 16 B, arranged activations
-// [4][K/64] x 16 B, row sums and row scales [R rounded to 4] each, and for ROT the rotated fp16
-// token + the rotation's transpose buffer.
-__host__ __device__ inline size_t code_bytes(int64_t R, int64_t K) { return (size_t)R * (size_t)(K / 4); }
-__host__ __device__ inline size_t rowacc_offset(int64_t R, int64_t K) { return code_bytes(R, K) + (size_t)K; }
-__host__ __device__ inline size_t sw_offset(int64_t R, int64_t K) {
-    return rowacc_offset(R, K) + (size_t)((R + 3) & ~3) * 4;
+// Shared memory after the static part: codes [R][K/64] x 16 B ([R][K/32] for 4-bit weights),
+// arranged activations (K bytes), row sums and row scales [R rounded to 4] each, and for ROT the
+// rotated fp16 token + the rotation's transpose buffer.
+__host__ __device__ inline size_t code_bytes(int64_t R, int64_t K, bool w4) {
+    return (size_t)R * (size_t)(w4 ? K / 2 : K / 4);
 }
-__host__ __device__ inline size_t xs_offset(int64_t R, int64_t K) { return sw_offset(R, K) + (size_t)((R + 3) & ~3) * 4; }
+__host__ __device__ inline size_t rowacc_offset(int64_t R, int64_t K, bool w4) { return code_bytes(R, K, w4) + (size_t)K; }
+__host__ __device__ inline size_t sw_offset(int64_t R, int64_t K, bool w4) {
+    return rowacc_offset(R, K, w4) + (size_t)((R + 3) & ~3) * 4;
+}
+__host__ __device__ inline size_t xs_offset(int64_t R, int64_t K, bool w4) {
+    return sw_offset(R, K, w4) + (size_t)((R + 3) & ~3) * 4;
+}
 
 template <bool ROT, int LOGB, int SET, typename OutT>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -144,15 +165,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ float sa_s;
     __shared__ float red[kActThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t KW = K / 16;
-    const int CPR = (int)(K / 64);  // 16-byte code groups per row
+    constexpr bool W4 = SET == kSetInt4;
+    const int64_t KW = K / 16;                    // 16-byte activation groups
+    const int64_t CW = K / (W4 ? 8 : 16);         // code words per row
+    const int CPR = (int)(K / (W4 ? 32 : 64));    // 16-byte code groups per row
+    constexpr int AG = W4 ? 2 : 4;                // activation groups per code group
     const int64_t R = (N + G - 1) / G;
     const int64_t r0 = (int64_t)blockIdx.x * N / G, r1 = (int64_t)(blockIdx.x + 1) * N / G;
     const int nrows = (int)(r1 - r0);
     const uint4* cs = reinterpret_cast<const uint4*>(smem);
-    uint4* as = reinterpret_cast<uint4*>(smem + code_bytes(R, K));
-    int* row_acc = reinterpret_cast<int*>(smem + rowacc_offset(R, K));
-    float* sw_s = reinterpret_cast<float*>(smem + sw_offset(R, K));
+    uint4* as = reinterpret_cast<uint4*>(smem + code_bytes(R, K, W4));
+    int* row_acc = reinterpret_cast<int*>(smem + rowacc_offset(R, K, W4));
+    float* sw_s = reinterpret_cast<float*>(smem + sw_offset(R, K, W4));
 
     // 1. Before the wait: the barrier, this CTA's codes in flight, its weight scales, the
     //    activations' lines into L2.
@@ -168,10 +192,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         sw_s[i] = __ldg(s_w + r0 + i);
     }
     __syncthreads();
-    const uint32_t bytes = (uint32_t)code_bytes(nrows, K);
+    const uint32_t bytes = (uint32_t)code_bytes(nrows, K, W4);
     if (tid == 0 && bytes) {
         tc::mbar_arrive_expect_tx(&bar, bytes);
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(codes + r0 * KW);
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(codes + r0 * CW);
         for (uint32_t off = 0; off < bytes; off += kPiece)
             bulk_g2s(smem + off, src + off, bytes - off < kPiece ? bytes - off : kPiece, &bar);
     }
@@ -188,14 +212,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     int qs = 0;
     if constexpr (ROT) {
         if (tid < kActThreads) {
-            __half* xs = reinterpret_cast<__half*>(smem + xs_offset(R, K));
-            float* tbuf = reinterpret_cast<float*>(smem + xs_offset(R, K) + (size_t)K * 2);
+            __half* xs = reinterpret_cast<__half*>(smem + xs_offset(R, K, W4));
+            float* tbuf = reinterpret_cast<float*>(smem + xs_offset(R, K, W4) + (size_t)K * 2);
             const float m = rotate_token_f16<LOGB, GroupSync<kActThreads>>(x, K, c, xs, tbuf, red);
             const float inv = m == 0.0f ? 0.0f : __fdiv_rn(7.0f, m);
             for (int g = tid; g < (int)KW; g += kActThreads) {
                 const uint4 v = m == 0.0f ? make_uint4(0u, 0u, 0u, 0u) : quant16(xs + 16 * g, inv);
                 if (blockIdx.x == 0 && q_out) *reinterpret_cast<uint4*>(q_out + 16 * g) = v;
-                as[(g & 3) * CPR + (g >> 2)] = arrange<SET>(v);
+                as[(g % AG) * CPR + g / AG] = arrange<SET>(v);
                 if constexpr (SET == kSetQift) qs = sum16(v, qs);
             }
             if (tid == 0) {
@@ -206,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     } else {
         for (int g = tid; g < (int)KW; g += kThreads) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(q) + g);
-            as[(g & 3) * CPR + (g >> 2)] = arrange<SET>(v);
+            as[(g % AG) * CPR + g / AG] = arrange<SET>(v);
             if constexpr (SET == kSetQift) qs = sum16(v, qs);
         }
         if (tid == 0) sa_s = __ldg(s_a);
@@ -231,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok && rg < RG) {
         uint4 a[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) a[u] = ch < CPR ? as[u * CPR + ch] : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < 4; ++u) a[u] = u < AG && ch < CPR ? as[u * CPR + ch] : make_uint4(0u, 0u, 0u, 0u);
         for (int row0 = rg; row0 < nrows; row0 += 4 * RG) {  // four independent rows per pass
             int v[4];
 #pragma unroll
@@ -261,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // 4. Epilogue: y = ((float)acc * s_w) * s_a.
     for (int t = tid; t < nrows; t += kThreads) {
-        const int acc = SET == kSetQift ? 2 * row_acc[t] - 3 * qsum : row_acc[t];
+        const int acc = SET == kSetQift ? 2 * row_acc[t] - 3 * qsum : (W4 ? row_acc[t] >> 4 : row_acc[t]);
         store_out<OutT>(y + r0 + t, __fmul_rn(__fmul_rn((float)acc, sw_s[t]), sa_s));
     }
 }
@@ -279,14 +303,14 @@ static int sm_count() {
 
 // Grid: one CTA per SM (two when the codes of one CTA would pass kMaxCodeBytes), never more
 // CTAs than rows.  Returns 0 when the matrix is too tall for this kernel.
-static int plan_grid(int64_t N, int64_t K, size_t extra_smem, size_t* smem) {
+static int plan_grid(int64_t N, int64_t K, size_t extra_smem, size_t* smem, bool w4) {
     if (N <= 0 || K <= 0 || K % 64 != 0 || K > 16384) return 0;
     const int sm = sm_count();
     for (int mult = 1; mult <= 2; ++mult) {
         const int64_t G = std::min<int64_t>(N, (int64_t)sm * mult);
         const int64_t R = (N + G - 1) / G;
-        if ((int64_t)code_bytes(R, K) > kMaxCodeBytes) continue;
-        const size_t bytes = xs_offset(R, K) + extra_smem;
+        if ((int64_t)code_bytes(R, K, w4) > kMaxCodeBytes) continue;
+        const size_t bytes = xs_offset(R, K, w4) + extra_smem;
         if (bytes > 200 * 1024) continue;
         *smem = bytes;
         return (int)G;
@@ -300,7 +324,7 @@ static cudaError_t launch(const __half* x, float c, const int8_t* q, const float
                           cudaStream_t s) {
     size_t smem = 0;
     const size_t extra = ROT ? (size_t)K * 2 + act_tbuf_bytes<LOGB>() : 0;
-    const int G = plan_grid(N, K, extra, &smem);
+    const int G = plan_grid(N, K, extra, &smem, SET == kSetInt4);
     if (!G) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem(one_token_kernel<ROT, LOGB, SET, OutT>, smem);
     if (e != cudaSuccess) return e;
@@ -325,6 +349,8 @@ static cudaError_t decode_by_set(const __half* x, float c, const uint32_t* codes
                                  int64_t N, int64_t K, OutT* y, int8_t* q_out, float* sa_out, cudaStream_t s) {
     if (set == kSetQift)
         return launch<true, LOGB, kSetQift, OutT>(x, c, nullptr, nullptr, codes, s_w, N, K, y, q_out, sa_out, s);
+    if (set == kSetInt4)
+        return launch<true, LOGB, kSetInt4, OutT>(x, c, nullptr, nullptr, codes, s_w, N, K, y, q_out, sa_out, s);
     return launch<true, LOGB, kSetPot, OutT>(x, c, nullptr, nullptr, codes, s_w, N, K, y, q_out, sa_out, s);
 }
 
@@ -354,7 +380,7 @@ static cudaError_t decode_by_block(const __half* x, int block, const uint32_t* c
 
 bool linear_one_token_supported(int64_t n_out, int64_t n_in) {
     size_t smem = 0;
-    return one::plan_grid(n_out, n_in, 0, &smem) != 0;
+    return one::plan_grid(n_out, n_in, 0, &smem, false) != 0;
 }
 
 // The warp-per-row GEMV (8 rows per 128-thread CTA, ~110 registers: four CTAs per SM) decodes
@@ -385,9 +411,9 @@ static size_t rotation_tbuf_bytes(int block) {
     }
 }
 
-bool decode_one_token_supported(int64_t n_out, int64_t n_in, int block) {
+bool decode_one_token_supported(int64_t n_out, int64_t n_in, int block, int set) {
     size_t smem = 0;
-    return one::plan_grid(n_out, n_in, (size_t)n_in * 2 + rotation_tbuf_bytes(block), &smem) != 0;
+    return one::plan_grid(n_out, n_in, (size_t)n_in * 2 + rotation_tbuf_bytes(block), &smem, set == kSetInt4) != 0;
 }
 
 cudaError_t launch_linear_one_token(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w,
