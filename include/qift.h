@@ -209,7 +209,8 @@ qift_status qift_decode_linear(const void* x, int64_t tokens, int64_t n_in, int3
 
 /* qift_device_error -- synchronise `stream`, then read and clear the device error word.
  * Returns QIFT_OK, QIFT_ERR_TIMEOUT (a bounded on-chip wait gave up; that call's output is
- * invalid) or QIFT_ERR_CUDA.  *detail (may be NULL) receives the raw word.  The word is one per
+ * invalid) or QIFT_ERR_CUDA (a CUDA error, or -- in the bounds-checked test build only -- a failed
+ * bounds check, bit 0x100 of the word).  *detail (may be NULL) receives the raw word.  The word is one per
  * device (the current one), not per stream or per call: a timeout of a kernel on any stream of
  * the device is reported to -- and cleared by -- whichever caller reads it first, so a caller
  * that runs work on several streams should synchronise them before reading it. */

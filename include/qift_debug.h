@@ -48,6 +48,18 @@ qift_status qift_debug_set_pdl(int32_t enable);
  * only the calls that thread makes. */
 qift_status qift_debug_set_linear_path(int32_t path);
 
+/* 1 in the bounds-checked build of the library (compiled with -DQIFT_CHECK, for tests), 0 in
+ * the normal build.  In the checked build every global index, bulk-copy range, tensor-map
+ * coordinate and tensor-memory address a kernel computes is tested against the extent its
+ * arguments imply; a failed test skips that access, sets bit 0x100 of the device error word
+ * (qift_device_error() then returns QIFT_ERR_CUDA with that bit in *detail) and keeps the source
+ * line of the first failure. */
+int32_t qift_debug_checked_build(void);
+
+/* Read and clear the source line of the first failed bounds check since the last call (0: none;
+ * always 0 in the normal build).  Call after qift_device_error() has synchronised the stream. */
+qift_status qift_debug_check_line(int32_t* line);
+
 #ifdef __cplusplus
 }
 #endif

@@ -545,6 +545,21 @@ def test_linear_each_kernel_family(path, name, T, N, K):
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
 
 
+@pytest.mark.parametrize("name", ["qift", "pot"])
+@pytest.mark.parametrize("N,K", [(5, 64), (37, 1088), (300, 2112), (130, 4160), (64, 6208), (257, 11008), (3, 32768)])
+def test_linear_one_token_gemv_partial_chunks(name, N, K):
+    # the warp-per-row GEMV stages the token in 2048-input chunks: rows of one partial chunk,
+    # and of several chunks with a partial last one, on the pinned family
+    qg.qift_debug_set_linear_path("gemv")
+    try:
+        for out_dtype in (torch.float16, torch.float32):
+            got, ref = _linear_case(name, 1, N, K, 5 * N + K, out_dtype)
+            u = np.uint16 if out_dtype == torch.float16 else np.uint32
+            assert np.array_equal(got.view(u), ref.view(u)), (name, N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+
+
 def test_prefill_with_unaligned_inputs_is_refused_not_slow():
     """Seventeen or more tokens run on the tensor cores only; an n_in they cannot take (not a
     multiple of 64) is refused, not sent to the CUDA-core GEMV.  Pinned to the GEMV the same call

@@ -18,7 +18,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqift.so")
+# QIFT_LIB_PATH selects another build of the same library -- the bounds-checked test build
+# (libqift_check.so, `python -m w2a4_gemm_b200.build --check`); by default the normal one.
+LIB_PATH = os.environ.get("QIFT_LIB_PATH") or os.path.join(_HERE, "libqift.so")
 
 QIFT_OK, QIFT_ERR_INVALID_ARG, QIFT_ERR_UNSUPPORTED, QIFT_ERR_CUDA, QIFT_ERR_TIMEOUT = range(5)
 QIFT_SET_QIFT, QIFT_SET_POT, QIFT_SET_STD, QIFT_SET_INT4 = 0, 1, 2, 3
@@ -57,6 +59,9 @@ def lib() -> C.CDLL:
         L.qift_debug_stall_next_one_token.argtypes = []
         L.qift_debug_set_linear_path.argtypes = [i32]
         L.qift_debug_set_pdl.argtypes = [i32]
+        L.qift_debug_check_line.argtypes = [C.POINTER(i32)]
+        L.qift_debug_checked_build.argtypes = []
+        L.qift_debug_checked_build.restype = i32
         L.qift_status_string.argtypes = [i32]
         L.qift_status_string.restype = C.c_char_p
         for name in ("qift_rotate", "qift_quantize_weights", "qift_rotate_quantize_weights",
@@ -65,7 +70,7 @@ def lib() -> C.CDLL:
                      "qift_linear", "qift_decode_linear",
                      "qift_device_error", "qift_debug_set_wait_limit", "qift_debug_stall_next_gemm",
                      "qift_debug_stall_next_one_token",
-                     "qift_debug_set_linear_path", "qift_debug_set_pdl"):
+                     "qift_debug_set_linear_path", "qift_debug_set_pdl", "qift_debug_check_line"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -340,6 +345,19 @@ def qift_device_error(stream=None) -> tuple[int, int]:
     detail = C.c_int32(0)
     st = lib().qift_device_error(_stream(stream), C.byref(detail))
     return st, detail.value
+
+
+def qift_debug_checked_build() -> bool:
+    """True when the loaded library is the bounds-checked test build."""
+    return bool(lib().qift_debug_checked_build())
+
+
+def qift_debug_check_line() -> int:
+    """Source line of the first failed bounds check since the last call (0: none; always 0 in
+    the normal build).  Read after qift_device_error(), which synchronises."""
+    line = C.c_int32(0)
+    _check(lib().qift_debug_check_line(C.byref(line)), "qift_debug_check_line")
+    return line.value
 
 
 def qift_debug_set_wait_limit(cycles: int) -> None:

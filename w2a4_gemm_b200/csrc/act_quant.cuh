@@ -89,7 +89,7 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
     __half2 amax2 = __float2half2_rn(0.0f);
     if constexpr (LOGB == 0) {
         for (int64_t i = (int64_t)tid * 8; i < K; i += kActThreads * 8) {
-            const uint4 t = *reinterpret_cast<const uint4*>(xt + i);
+            const uint4 t = QIFT_CK_RANGE(i, 8, K) ? *reinterpret_cast<const uint4*>(xt + i) : make_uint4(0u, 0u, 0u, 0u);
             *reinterpret_cast<uint4*>(xs + i) = t;
             const __half2* h = reinterpret_cast<const __half2*>(&t);
 #pragma unroll
@@ -100,7 +100,12 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
         const int lo = tid & 15, hi = tid >> 4;
         for (int64_t seg = 0; seg < K / 4096; ++seg) {
             float v[16];
-            load_contig<16>(xt + seg * 4096 + tid * 16, v);
+            if (QIFT_CK_RANGE(seg * 4096 + tid * 16, 16, K)) {
+                load_contig<16>(xt + seg * 4096 + tid * 16, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+            }
             reg_stages<16>(v);  // h = 1 .. 8
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
@@ -134,7 +139,7 @@ __device__ __forceinline__ float rotate_token_f16(const InT* __restrict__ xt, in
             const int64_t seg = p + seg_local;
             const bool active = seg < nseg;
             float v[S::E];
-            if (active) {
+            if (active && QIFT_CK_RANGE(seg * S::B + ts * S::E, S::E, K)) {
                 load_contig<S::E>(xt + seg * S::B + ts * S::E, v);
             } else {
 #pragma unroll

@@ -264,7 +264,24 @@ qift_status qift_device_error(void* stream, int32_t* detail) {
     if (qift::read_and_clear_one_token_error(&word1) != cudaSuccess) return QIFT_ERR_CUDA;
     word |= word1;
     if (detail) *detail = word;
+    if (word & 0x100) return QIFT_ERR_CUDA;  // a failed bounds check (checked build only)
     return word ? QIFT_ERR_TIMEOUT : QIFT_OK;
+}
+
+qift_status qift_debug_check_line(int32_t* line) {
+    if (!line) return QIFT_ERR_INVALID_ARG;
+    int v = 0;
+    if (qift::read_and_clear_check_line(&v) != cudaSuccess) return QIFT_ERR_CUDA;
+    *line = v;
+    return QIFT_OK;
+}
+
+int32_t qift_debug_checked_build(void) {
+#ifdef QIFT_CHECK
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 qift_status qift_debug_set_wait_limit(int64_t cycles) {

@@ -11,6 +11,39 @@
 
 namespace qift {
 
+// Bounds-checked build (-DQIFT_CHECK, a separate library for tests): QIFT_CK(cond) tests an
+// index, copy range, tensor-map coordinate or tensor-memory address against the extent the
+// kernel's own arguments imply.  A failed test sets bit 0x100 of the device error word, keeps
+// the first failing source line, and yields false, so the guarded access is skipped: no trap,
+// and no thread leaves code that others synchronise with.  In the normal build QIFT_CK(cond)
+// is the constant true and cond is not evaluated.
+// The recorded site is file_tag(__FILE__) * 100000 + __LINE__: the tag is an FNV-1a hash of
+// the file's base name, modulo 1000.
+__host__ __device__ constexpr uint32_t fnv1a_tail(const char* s, uint32_t h) {
+    return *s ? fnv1a_tail(s + 1, (h ^ (uint32_t)(unsigned char)*s) * 16777619u) : h;
+}
+__host__ __device__ constexpr const char* base_name(const char* s, const char* last) {
+    return *s ? base_name(s + 1, *s == '/' ? s + 1 : last) : last;
+}
+__host__ __device__ constexpr int file_tag(const char* path) {
+    return (int)(fnv1a_tail(base_name(path, path), 2166136261u) % 1000u);
+}
+#ifdef QIFT_CHECK
+extern __device__ int g_qift_error;
+extern __device__ int g_qift_check_line;
+__device__ __noinline__ inline bool check_fail(int site) {
+    atomicOr(&g_qift_error, 0x100);
+    atomicCAS(&g_qift_check_line, 0, site);
+    return false;
+}
+#define QIFT_CK(cond) ((cond) || ::qift::check_fail(::qift::file_tag(__FILE__) * 100000 + __LINE__))
+#else
+#define QIFT_CK(cond) true
+#endif
+// [off, off + len) inside [0, extent)
+#define QIFT_CK_RANGE(off, len, extent) \
+    QIFT_CK((int64_t)(off) >= 0 && (int64_t)(off) + (int64_t)(len) <= (int64_t)(extent))
+
 constexpr int kSetQift = 0;
 constexpr int kSetPot = 1;
 constexpr int kSetStd = 2;

@@ -71,8 +71,9 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
 #pragma unroll
             for (int j = 0; j < J; ++j) {
                 const int64_t wi = base + 4 * lane + 128 * j;
-                const uint4 v = (r < nr && wi + 4 <= KW) ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
-                                                         : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 v = (r < nr && wi + 4 <= KW && QIFT_CK_RANGE((row0 + r) * KW + wi, 4, N * KW))
+                                    ? ldg_stream_v4(codes + (row0 + r) * KW + wi)
+                                    : make_uint4(0u, 0u, 0u, 0u);
                 if constexpr (W4) {
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
     griddep_wait();
     float sw[RMAX];
 #pragma unroll
-    for (int r = 0; r < RMAX; ++r) sw[r] = r < nr ? __ldg(s_w + row0 + r) : 0.0f;
+    for (int r = 0; r < RMAX; ++r) sw[r] = r < nr && QIFT_CK_RANGE(row0 + r, 1, N) ? __ldg(s_w + row0 + r) : 0.0f;
 
     // 2. rotation + INT4 of every token, identical arithmetic to qift_quantize_acts.
     for (int t = 0; t < TC; ++t) {
@@ -106,7 +107,8 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
             const float inv = m == 0.0f ? 0.0f : __fdiv_rn(7.0f, m);
             for (int64_t i = (int64_t)tid * 16; i < K; i += kActThreads * 16) {
                 const uint4 v = m == 0.0f ? make_uint4(0u, 0u, 0u, 0u) : quant16(xs + i, inv);
-                if (blockIdx.x == 0 && q_out) *reinterpret_cast<uint4*>(q_out + (int64_t)t * K + i) = v;
+                if (blockIdx.x == 0 && q_out && QIFT_CK_RANGE((int64_t)t * K + i, 16, (int64_t)T * K))
+                    *reinterpret_cast<uint4*>(q_out + (int64_t)t * K + i) = v;
                 if constexpr (W4) {
                     *reinterpret_cast<uint4*>(qt + i) = v;  // natural order
                 } else {
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kActThreads) decode_kernel(const __half* __res
         for (int t = 0; t < TC; ++t) {
             int sum = __reduce_add_sync(0xffffffffu, acc[r][t]);
             if constexpr (W4) sum >>= 4;  // exact: every product was 16 x level x q
-            if (lane == ((r * TC + t) & 31) && t < T) {
+            if (lane == ((r * TC + t) & 31) && t < T && QIFT_CK_RANGE((int64_t)t * N + row0 + r, 1, (int64_t)T * N)) {
                 const float v = __fmul_rn(__fmul_rn((float)sum, sw[r]), sa_s[t]);
                 store_out<OutT>(y + (int64_t)t * N + row0 + r, v);
             }

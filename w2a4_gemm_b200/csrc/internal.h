@@ -116,6 +116,10 @@ bool pdl_enabled();  // programmatic dependent launch for the decode kernels (de
 void debug_set_gemm_wait_limit(long long cycles);
 void debug_stall_next_gemm();
 
+// Bounds-checked build: read and clear the source line of the first failed check (0: none, and
+// always 0 in the normal build).
+cudaError_t read_and_clear_check_line(int* line);
+
 // Synchronous read-and-clear of the device error word set by bounded on-chip waits.
 cudaError_t read_and_clear_device_error(int* word);
 

@@ -20,6 +20,9 @@
 namespace qift {
 
 __device__ int g_qift_error = 0;  // QIFT_ERR_TIMEOUT-style bits, read by qift_device_error()
+#ifdef QIFT_CHECK
+__device__ int g_qift_check_line = 0;  // bounds-checked build: source line of the first failed check
+#endif
 
 // =====================================================================================
 // CTA-pair GEMM, persistent.  A cluster of two CTAs on two SMs computes 256-weight-row x
@@ -236,13 +239,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const bool second = !W4 && kb * BK + 128 < K;
                     if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_ctas * (second ? 2u : 1u) * ACT_HALF);
                     tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
-                    if (has_act) {
+                    // tensor-map coordinates: x a 16-byte multiple inside the row, y inside the matrix
+                    if (has_act && QIFT_CK((kb * BKI) % 16 == 0 && kb * BKI < K && tb >= 0 && tb < T)) {
                         tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BKI, tb);
                         if (second)
                             tc::tma_load_2d_pair(sm.act + s * ACT_BYTES + ACT_HALF, &tmap_x, full0 + 8 * s,
                                                  kb * BK + 128, tb);
                     }
-                    if (has_cod)
+                    if (has_cod && QIFT_CK(kb * 16 * (W4 ? 8 : 16) < K && tl.n0 >= 0 && tl.n0 < N))
                         tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * 16, tl.n0);
                 }
             }
@@ -275,6 +279,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint64_t d = desc0 + (uint64_t)((s * ACT_BYTES) >> 4);
                     const uint64_t d2 = d + (uint64_t)(ACT_HALF >> 4);
                     const uint32_t a = tmem + A_COL + (BK / 4) * s;
+                    // the A stage's columns and the accumulator's lie inside the allocation
+                    if (!QIFT_CK(A_COL + (BK / 4) * (s + 1) <= TMEM_COLS && ACC_COL + BNT <= A_COL)) {
+                        ok = false;
+                        break;
+                    }
                     tc::mma_i8_ts_pair(tmem + ACC_COL, a, d, idesc, kb != 0 ? 1u : 0u);
 #pragma unroll
                     for (int k = 1; k < 4; ++k) tc::mma_i8_ts_pair(tmem + ACC_COL, a + 8 * k, d + 2 * k, idesc, 1u);
@@ -309,6 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       (rank != 0 || wait_fast(&sm.full[s], ph, sm.abort, wait_limit));
             if (!__all_sync(0xffffffffu, ok)) break;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + A_COL + (BK / 4) * s;
+            if (!QIFT_CK(quarter == (warp & 3) && A_COL + (BK / 4) * (s + 1) <= TMEM_COLS)) break;
             const uint8_t* crow = sm.cod + s * COD_BYTES + r * 64;
             tc::tc_fence_after();
             if constexpr (W4) {  // 128 inputs (sixteen code words) in one tensor-memory store
@@ -384,6 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const int cl0 = cgrp * CPW + cc * 32;  // column within the pass
                         const int c0 = p * CPP + cl0;         // column within the tile
                         uint32_t acc[32];
+                        if (!QIFT_CK(c0 + 32 <= BNT && quarter == (warp & 3))) continue;
                         tc::tmem_ld_32x32b_x32(tmem + ((uint32_t)(quarter * 32) << 16) + ACC_COL + c0, acc);
                         tc::tmem_ld_wait();
                         if constexpr (sizeof(OutT) == 2) {
@@ -433,12 +444,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 for (int tt = 0; tt < 2 && t + tt < T; ++tt) {
                                     const uint32_t* w = tt ? hi : lo;
                                     OutT* dst = y + (int64_t)(t + tt) * N + nn;
+                                    const int64_t off = (int64_t)(t + tt) * N + nn;
                                     if (vec_ok && nn + EPP <= N) {
-                                        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                                        if (QIFT_CK_RANGE(off, EPP, (int64_t)T * N))
+                                            *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
                                     } else {
                                         const __half* hv = reinterpret_cast<const __half*>(w);
                                         for (int e = 0; e < EPP; ++e)
-                                            if (nn + e < N) dst[e] = hv[e];
+                                            if (nn + e < N && QIFT_CK_RANGE(off + e, 1, (int64_t)T * N)) dst[e] = hv[e];
                                     }
                                 }
                             }
@@ -451,11 +464,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             if (t < T) {
                                 OutT* dst = y + (int64_t)t * N + nn;
                                 const OutT* src = stg + j * BMW + sub * EPP;
+                                const int64_t off = (int64_t)t * N + nn;
                                 if (vec_ok && nn + EPP <= N) {
-                                    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                                    if (QIFT_CK_RANGE(off, EPP, (int64_t)T * N))
+                                        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
                                 } else {
                                     for (int e = 0; e < EPP; ++e)
-                                        if (nn + e < N) dst[e] = src[e];
+                                        if (nn + e < N && QIFT_CK_RANGE(off + e, 1, (int64_t)T * N)) dst[e] = src[e];
                                 }
                             }
                         }
@@ -569,6 +584,18 @@ void debug_set_gemm_wait_limit(long long cycles) {
     gemm_pair::g_wait_limit = cycles > 0 ? cycles : gemm_pair::kWaitCycles;
 }
 void debug_stall_next_gemm() { gemm_pair::g_stall_next = true; }
+
+cudaError_t read_and_clear_check_line(int* line) {
+    *line = 0;
+#ifdef QIFT_CHECK
+    cudaError_t e = cudaMemcpyFromSymbol(line, g_qift_check_line, sizeof(int));
+    if (e != cudaSuccess || *line == 0) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_qift_check_line, &zero, sizeof(int));
+#else
+    return cudaSuccess;
+#endif
+}
 
 cudaError_t read_and_clear_device_error(int* word) {
     int v = 0;

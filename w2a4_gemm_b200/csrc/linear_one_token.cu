@@ -189,11 +189,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     for (int i = tid; i < nrows; i += kThreads) {
         row_acc[i] = 0;
-        sw_s[i] = __ldg(s_w + r0 + i);
+        sw_s[i] = QIFT_CK_RANGE(r0 + i, 1, N) ? __ldg(s_w + r0 + i) : 0.0f;
     }
     __syncthreads();
     const uint32_t bytes = (uint32_t)code_bytes(nrows, K, W4);
-    if (tid == 0 && bytes) {
+    if (tid == 0 && bytes && QIFT_CK_RANGE(r0 * CW * 4, bytes, N * CW * 4) && QIFT_CK(bytes % 16 == 0) &&
+        QIFT_CK(code_bytes(R, K, W4) >= bytes)) {
         tc::mbar_arrive_expect_tx(&bar, bytes);
         const uint8_t* src = reinterpret_cast<const uint8_t*>(codes + r0 * CW);
         for (uint32_t off = 0; off < bytes; off += kPiece)
@@ -218,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float inv = m == 0.0f ? 0.0f : __fdiv_rn(7.0f, m);
             for (int g = tid; g < (int)KW; g += kActThreads) {
                 const uint4 v = m == 0.0f ? make_uint4(0u, 0u, 0u, 0u) : quant16(xs + 16 * g, inv);
-                if (blockIdx.x == 0 && q_out) *reinterpret_cast<uint4*>(q_out + 16 * g) = v;
+                if (blockIdx.x == 0 && q_out && QIFT_CK_RANGE(16 * (int64_t)g, 16, K))
+                    *reinterpret_cast<uint4*>(q_out + 16 * g) = v;
                 as[(g % AG) * CPR + g / AG] = arrange<SET>(v);
                 if constexpr (SET == kSetQift) qs = sum16(v, qs);
             }
@@ -229,7 +231,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else {
         for (int g = tid; g < (int)KW; g += kThreads) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(q) + g);
+            const uint4 v = QIFT_CK_RANGE(16 * (int64_t)g, 16, K) ? __ldg(reinterpret_cast<const uint4*>(q) + g)
+                                                                   : make_uint4(0u, 0u, 0u, 0u);
             as[(g % AG) * CPR + g / AG] = arrange<SET>(v);
             if constexpr (SET == kSetQift) qs = sum16(v, qs);
         }
@@ -286,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // 4. Epilogue: y = ((float)acc * s_w) * s_a.
     for (int t = tid; t < nrows; t += kThreads) {
         const int acc = SET == kSetQift ? 2 * row_acc[t] - 3 * qsum : (W4 ? row_acc[t] >> 4 : row_acc[t]);
-        store_out<OutT>(y + r0 + t, __fmul_rn(__fmul_rn((float)acc, sw_s[t]), sa_s));
+        if (QIFT_CK_RANGE(r0 + t, 1, N)) store_out<OutT>(y + r0 + t, __fmul_rn(__fmul_rn((float)acc, sw_s[t]), sa_s));
     }
 }
 

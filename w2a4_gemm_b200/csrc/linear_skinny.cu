@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
         lo = make_uint4(0u, 0u, 0u, 0u);
         hi = make_uint4(0u, 0u, 0u, 0u);
         if (wi + 4 <= KW) {
-            if (r_lo < N) lo = ldg_stream_v4(codes + r_lo * KW + wi);
-            if (r_hi < N) hi = ldg_stream_v4(codes + r_hi * KW + wi);
+            if (r_lo < N && QIFT_CK_RANGE(r_lo * KW + wi, 4, N * KW)) lo = ldg_stream_v4(codes + r_lo * KW + wi);
+            if (r_hi < N && QIFT_CK_RANGE(r_hi * KW + wi, 4, N * KW)) hi = ldg_stream_v4(codes + r_hi * KW + wi);
         }
     };
 
@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
             const int t = i / groups, G = i - t * groups;
             const int64_t k = (int64_t)rank * KS + (int64_t)G * 16;  // input index of group G
             a[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < TP * groups && t < T && k + 16 <= K) a[u] = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
+            if (i < TP * groups && t < T && k + 16 <= K && QIFT_CK_RANGE((int64_t)t * K + k, 16, (int64_t)T * K))
+                a[u] = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -237,10 +238,12 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
     for (int i = threadIdx.x; i < rows_per * TP; i += THREADS) {
         const int t = i / rows_per, rl = rank * rows_per + (i - t * rows_per);
         int sum = 0;
-        for (int p = 0; p < C; ++p) sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
+        for (int p = 0; p < C; ++p)
+            if (QIFT_CK(p < (int)cluster.num_blocks() && t * RBP + rl < TP * RBP))
+                sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
         if constexpr (W4) sum >>= 4;  // exact: every product was 16 x level x q
         const int64_t n = (int64_t)row_block * RB + rl;
-        if (t < T && n < N) {
+        if (t < T && n < N && QIFT_CK_RANGE((int64_t)t * N + n, 1, (int64_t)T * N)) {
             const float v = __fmul_rn(__fmul_rn((float)sum, sw_s[rl]), sa_s[t]);
             store_y<OutT>(y + (int64_t)t * N + n, v);
         }

@@ -52,8 +52,9 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
     auto load_codes = [&](int64_t g) {
 #pragma unroll
         for (int r = 0; r < R; ++r)
-            cw[r] = (row0 + r < N && g < KG) ? ldg_stream_v4(codes + (row0 + r) * KW + 4 * g)
-                                             : make_uint4(0u, 0u, 0u, 0u);
+            cw[r] = (row0 + r < N && g < KG && QIFT_CK_RANGE((row0 + r) * KW + 4 * g, 4, N * KW))
+                        ? ldg_stream_v4(codes + (row0 + r) * KW + 4 * g)
+                        : make_uint4(0u, 0u, 0u, 0u);
     };
     load_codes(lane);
     griddep_launch_dependents();
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
 #pragma unroll
         for (int t = 0; t < TC; ++t) {
             uint4 a0 = make_uint4(0u, 0u, 0u, 0u), a1 = a0;
-            if (t0 + t < T) {
+            if (t0 + t < T && QIFT_CK_RANGE((t0 + t) * K + 32 * g, 32, T * K)) {
                 const uint4* src = reinterpret_cast<const uint4*>(q + (t0 + t) * K + 32 * g);
                 a0 = __ldg(src);
                 a1 = __ldg(src + 1);
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kWarps * 32) w4_gemv_kernel(const int8_t* __re
         for (int t = 0; t < TC; ++t) {
             const int sum = __reduce_add_sync(0xffffffffu, acc[r][t]) >> 4;  // exact: a multiple of 16
             const int64_t n = row0 + r, tt = t0 + t;
-            if (lane == ((r * TC + t) & 31) && n < N && tt < T)
+            if (lane == ((r * TC + t) & 31) && n < N && tt < T && QIFT_CK_RANGE(tt * N + n, 1, T * N))
                 store_out<OutT>(y + tt * N + n, __fmul_rn(__fmul_rn((float)sum, __ldg(s_w + n)), __ldg(s_a + tt)));
         }
     }

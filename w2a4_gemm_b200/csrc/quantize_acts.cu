@@ -37,6 +37,7 @@ __global__ void __launch_bounds__(kActThreads) quant_acts_kernel(const __half* _
     int8_t* qt = q + token * (PACK ? K / 2 : K);
     if (m == 0.0f) {
         for (int64_t i = (int64_t)tid * 16; i < K; i += kActThreads * 16) {
+            if (!QIFT_CK_RANGE(i, 16, K)) continue;
             if constexpr (PACK) *reinterpret_cast<uint2*>(qt + i / 2) = make_uint2(0u, 0u);
             else *reinterpret_cast<uint4*>(qt + i) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -45,6 +46,7 @@ __global__ void __launch_bounds__(kActThreads) quant_acts_kernel(const __half* _
     }
     const float inv = __fdiv_rn(7.0f, m);
     for (int64_t i = (int64_t)tid * 16; i < K; i += kActThreads * 16) {
+        if (!QIFT_CK_RANGE(i, 16, K)) continue;
         if constexpr (PACK) *reinterpret_cast<uint2*>(qt + i / 2) = pack_int4_16(quant16(xs + i, inv));
         else *reinterpret_cast<uint4*>(qt + i) = quant16(xs + i, inv);
     }
@@ -72,6 +74,7 @@ __global__ void __launch_bounds__(kActThreads) dequant_kv_kernel(const uint8_t* 
     const uint8_t* pt = packed + token * (K / 2);
     __half* ot = out + token * K;
     for (int64_t i = (int64_t)tid * 16; i < K; i += kActThreads * 16) {
+        if (!QIFT_CK_RANGE(i, 16, K)) continue;
         const uint2 p = *reinterpret_cast<const uint2*>(pt + i / 2);
         float v[16];
 #pragma unroll
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(kActThreads) dequant_kv_kernel(const uint8_t* 
         __syncthreads();
         rotate_token_f16<LOGB, CtaSync, float>(xf, K, c, xs, tbuf, red);
         for (int64_t i = (int64_t)tid * 8; i < K; i += kActThreads * 8)
-            *reinterpret_cast<uint4*>(ot + i) = *reinterpret_cast<const uint4*>(xs + i);
+            if (QIFT_CK_RANGE(i, 8, K)) *reinterpret_cast<uint4*>(ot + i) = *reinterpret_cast<const uint4*>(xs + i);
     }
 }
 

@@ -196,7 +196,8 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
         for (int r = 0; r < rows; ++r) {
             const float* wr = w + (row0 + r) * K;
             for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4)
-                *reinterpret_cast<float4*>(ws + r * K + i) = *reinterpret_cast<const float4*>(wr + i);
+                if (QIFT_CK_RANGE((row0 + r) * K + i, 4, n_out * K))
+                    *reinterpret_cast<float4*>(ws + r * K + i) = *reinterpret_cast<const float4*>(wr + i);
         }
         __syncthreads();
         fwht_rows_in_smem(ws, rows, (int)K, logb, c);
@@ -210,11 +211,11 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
         if (r < rows) {
             const float* wr = w + (row0 + r) * K;
             for (int64_t i = (int64_t)tid * 4; i < K; i += nthr * 4) {
-                float4 v;
+                float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 if constexpr (ROT) {
                     v = *reinterpret_cast<const float4*>(ws + r * K + i);
                 } else {
-                    v = *reinterpret_cast<const float4*>(wr + i);
+                    if (QIFT_CK_RANGE((row0 + r) * K + i, 4, n_out * K)) v = *reinterpret_cast<const float4*>(wr + i);
                     *reinterpret_cast<float4*>(ws + r * K + i) = v;
                 }
                 if constexpr (SET == kSetAsym) {
@@ -319,9 +320,9 @@ __global__ void __launch_bounds__(1024) quant_weights_kernel(const float* __rest
                 word |= enc.code(v.z) << shift(4 * v4 + 2);
                 word |= enc.code(v.w) << shift(4 * v4 + 3);
             }
-            crow[j] = word;
+            if (QIFT_CK_RANGE((row0 + r) * (K / CPW) + j, 1, n_out * (K / CPW))) crow[j] = word;
         }
-        if (tid == 0) {
+        if (tid == 0 && QIFT_CK_RANGE(row0 + r, 1, n_out)) {
             scales[row0 + r] = SET == kSetQift ? __fmul_rn(sr, 0.5f) : sr;
             if constexpr (SET == kSetAsym) zeros[row0 + r] = zc[r * kQwMaxG + b];
             if (row_mse) row_mse[row0 + r] = __ddiv_rn(mse[r * kQwMaxG + b], (double)K);

@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(const T* x, T* y,
     const bool active = seg < n_segments;
 
     float v[S::E];
-    if (active) {
+    if (active && QIFT_CK_RANGE(seg * S::B + ts * S::E, S::E, n_segments * S::B)) {
         load_contig<S::E>(x + seg * S::B + ts * S::E, v);
     } else {
 #pragma unroll
@@ -37,7 +37,9 @@ __global__ void __launch_bounds__(kRotThreads) rotate_kernel(const T* x, T* y,
     if (active) {
         T* base = y + seg * S::B + ts * S::R;
 #pragma unroll
-        for (int j = 0; j < S::W; ++j) store_contig<S::R>(base + j * S::COL, out[j]);
+        for (int j = 0; j < S::W; ++j)
+            if (QIFT_CK_RANGE(seg * S::B + ts * S::R + j * S::COL, S::R, n_segments * S::B))
+                store_contig<S::R>(base + j * S::COL, out[j]);
     }
 }
 
