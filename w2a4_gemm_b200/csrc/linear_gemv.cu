@@ -194,9 +194,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv1_kernel(const int8_t* __
 #pragma unroll
     for (int r = 0; r < R; ++r) sw[r] = row0 + r < N ? __ldg(s_w + row0 + r) : 0.0f;
     const float sa = __ldg(s_a);
-    // Thread t reads word t (+ 128 per pass), coalesced, and stores it at its slot.  (Filling the
-    // slots in order instead -- conflict-free stores, reads 64 bytes apart -- measured slower:
-    // 2.34 against 2.02 us per launch at 4096 x 4096.)
+    // Thread t reads word t (+ 128 per pass), coalesced, and stores it at its slot (a 4-way
+    // bank conflict on the stores).  Measured slower: filling the slots in order with reads 64
+    // bytes apart (2.34 against 2.02 us per launch at 4096 x 4096), and conflict-free stores
+    // from a lane permutation inside each 32-word group (2.18 us).
     for (int i = threadIdx.x; i < (int)KW; i += kGemvWarps * 32) {
         uint32_t p[4];
         permute_acts(QIFT_CK_RANGE(16 * (int64_t)i, 16, K) ? __ldg(reinterpret_cast<const uint4*>(q) + i)
