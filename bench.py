@@ -70,11 +70,11 @@ def peaks():
 # as null.  `scale` converts the captured launch to the benchmarked one when the shapes differ
 # (traffic grows in proportion to the weights processed).
 PROFILED_TRAFFIC = {
-    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="7072e2cc258b4f58", bytes=4231168 + 0,
+    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="87eab3d8c0a24955", bytes=4225536 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
-    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="0401423015962d76",
-                    bytes=19752192 + 1284864, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
-    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="efcfee8669e604e6", bytes=14854144 + 0,
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="83bc35be637da8d0",
+                    bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="fc3be88d2dbf2100", bytes=14853888 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
     "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="7caa8a2d0ba3cce3",
                     bytes=67147776 + 1114368, scale=14336 * 4096 / (4096 * 4096),
