@@ -76,8 +76,8 @@ PROFILED_TRAFFIC = {
                     bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
     "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="fc3be88d2dbf2100", bytes=14853888 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
-    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="7caa8a2d0ba3cce3",
-                    bytes=67147776 + 1114368, scale=14336 * 4096 / (4096 * 4096),
+    "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="00f7bc2d84fdc9a9",
+                    bytes=67153920 + 1506816, scale=14336 * 4096 / (4096 * 4096),
                     profile="profiles/quant_weights_kernel_q_proj_4096x4096.md"),
 }
 
