@@ -464,7 +464,7 @@ def run_ours(args, rank, world):
         "a5_linear": linear_stage(torch, qg, st, L0, pk, reps, STAGE_REPLAYS, T, out_b),
     }
     lin_b = stages["a5_linear"]["bytes"]
-    if T <= 4 and K0 % 64 == 0 and K0 <= 16384 and wl.levelset in ("qift", "pot"):
+    if T <= 4 and K0 % 64 == 0 and K0 <= 16384 and wl.levelset in ("qift", "pot", "int4"):
         f_fn = lambda i: qg.qift_decode_linear(L0["x"][i % copies], wl.a_block, L0["codes"][i % copies],
                                                L0["s_w"][i % copies], wl.levelset, st.out_dt,
                                                out=L0["y"][i % copies])

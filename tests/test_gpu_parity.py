@@ -288,6 +288,13 @@ def test_linear_w4_extreme_accumulators():
         finally:
             qg.qift_debug_set_linear_path("auto")
         assert np.array_equal(host(gy), y), pin
+    # one token (the one-token kernel splits every code of its chunk before the wait)
+    for t in range(T):
+        y1, acc1 = oracle.linear_w4(q[t:t + 1], s_a[t:t + 1], codes, s_w, np.float32)
+        assert np.abs(acc1).max() == (49 * K if t < 2 else 0)  # token 2 alternates +-7: zero sum
+        gy = qg.qift_linear(dev(q[t:t + 1]), dev(s_a[t:t + 1]), dev(codes.view(np.int32)), dev(s_w), "int4",
+                            torch.float32)
+        assert np.array_equal(host(gy), y1), t
 
 
 @pytest.mark.parametrize("pin", ["auto", "gemm_pair"])
