@@ -8,14 +8,16 @@
 // Work split.  A thread-block cluster of C CTAs shares one block of 128 output rows; CTA r of
 // the cluster owns the K slice [r*KS, (r+1)*KS).  Each 16-row group of the block is owned by
 // one warp, or by two warps taking alternate 256-input chunks when the grid leaves an SM per
-// CTA (more warps in flight per SM; their int32 partials are added in shared memory).  The CTA
+// CTA (more warps in flight per SM).  The CTA
 // stages its slice of every token's int8 activations once in shared memory, permuted per
 // 16-byte group to the decode order, so the weights never touch shared memory: a lane loads
 // 16 bytes (4 words = 64 codes) of each of its two rows, decodes a word into four int8x4
 // registers with two masks, two shifts and four byte permutes against the level table, and
-// those registers ARE the A fragments of mma.m16n8k32 (s8 x s8 -> s32).  Partial int32 sums
-// of the C CTAs are added through distributed shared memory (exact, order-free), and the
-// cluster's CTAs each finish 128/C rows with the fp32 epilogue.  No global scratch.
+// those registers ARE the A fragments of mma.m16n8k32 (s8 x s8 -> s32).  Each warp pushes its
+// partial int32 sums into the shared memory of the cluster CTA that finishes those rows
+// (distributed shared memory); after one cluster barrier every CTA adds the partials it
+// received (exact, order-free) and finishes 128/C rows with the fp32 epilogue.  No global
+// scratch.
 //
 // Fragment bookkeeping (g = lane/4, q = lane%4).  For chunk c (16 words of a row) and sub-step
 // j = 0..3, thread q handles word w = 16c + 4q + j of rows g and g+8; decode_word gives
@@ -46,7 +48,6 @@ constexpr int ROW_WARPS = 8;                    // warps along the rows: 16 rows
 constexpr int RB = ROW_WARPS * 16;              // output rows per cluster
 constexpr int CHUNK_WORDS = 16;  // 256 K values per chunk
 constexpr int PF = 4;            // chunks of codes in flight per lane
-constexpr int RBP = RB + 4;      // padded row stride of the partial sums (conflict-free writes)
 
 __device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -81,13 +82,18 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
     extern __shared__ __align__(16) uint8_t smem[];
     const int S = KS + 64;                            // token row stride (== 64 mod 128)
     uint8_t* acts = smem;                             // TP x S bytes
-    int* part = reinterpret_cast<int*>(smem + TP * S);  // [TP][RBP] int32 partial sums
-    float* sa_s = reinterpret_cast<float*>(part + TP * RBP);  // [TP] activation scales
-    float* sw_s = sa_s + TP;                                    // [RB] weight scales of the block
-
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
+    // The CTA finishes RB/C rows of the block; C is a power of two, so RB/C is too.
+    const int lg_rows = 7 - (__ffs(C) - 1);  // log2(RB / C), RB = 128
+    const int rows_per = 1 << lg_rows;
+    const int RPS = rows_per + 4;            // row stride of the partial sums (conflict-free writes)
+    // part[s][token][row]: the int32 partial sums this CTA's rows receive, one slot s per source
+    // CTA of the cluster and K parity of its warps.
+    int* part = reinterpret_cast<int*>(smem + TP * S);
+    float* sa_s = reinterpret_cast<float*>(part + KSPLIT * C * TP * RPS);  // [TP] activation scales
+    float* sw_s = sa_s + TP;                                                // [RB] weight scales of the block
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, qd = lane & 3;
     const int row_block = blockIdx.x / C;
@@ -111,6 +117,10 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
         }
     };
 
+    // Announce that this CTA has started; the matching wait below, before the first write into a
+    // peer's shared memory, guarantees every peer exists by then.
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+
     // Weights do not depend on the previous kernel: start streaming them before waiting.  A
     // ring of PF chunks per lane keeps PF KB of codes per warp in flight.
     uint4 buf[PF][2];
@@ -120,31 +130,43 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
     griddep_wait();
 
     // Stage this CTA's K slice of every token, permuted to the decode order (eight loads in
-    // flight per thread before any is used), and the scales the epilogue needs.
+    // flight per thread before any is used), and the scales the epilogue needs.  Element i is
+    // group G = i % groups of token t = i / groups; a thread steps its (t, G) by THREADS with one
+    // division up front.
     const int groups = KS / 16;
+    const int dt = THREADS / groups, dg = THREADS - dt * groups;
+    int t_i = (int)threadIdx.x / groups, g_i = (int)threadIdx.x - t_i * groups;
+    const uint8_t* q_slice = reinterpret_cast<const uint8_t*>(q) + (int64_t)rank * KS;
+    const int64_t rest = ((int64_t)K - (int64_t)rank * KS) / 16;  // groups of the slice inside the row
+    const int g_lim = rest < groups ? (int)rest : groups;
     for (int i0 = 0; i0 < TP * groups; i0 += 8 * THREADS) {
         uint4 a[8];
+        int tt[8], gg[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * THREADS + threadIdx.x;
-            const int t = i / groups, G = i - t * groups;
-            const int64_t k = (int64_t)rank * KS + (int64_t)G * 16;  // input index of group G
+            tt[u] = t_i;
+            gg[u] = g_i;
             a[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < TP * groups && t < T && k + 16 <= K && QIFT_CK_RANGE((int64_t)t * K + k, 16, (int64_t)T * K))
-                a[u] = __ldg(reinterpret_cast<const uint4*>(q + (int64_t)t * K + k));
+            if (t_i < T && g_i < g_lim &&
+                QIFT_CK_RANGE((int64_t)t_i * K + (int64_t)rank * KS + 16 * g_i, 16, (int64_t)T * K))
+                a[u] = __ldg(reinterpret_cast<const uint4*>(q_slice + (int64_t)t_i * K + 16 * g_i));
+            t_i += dt;
+            g_i += dg;
+            if (g_i >= groups) {
+                g_i -= groups;
+                ++t_i;
+            }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * THREADS + threadIdx.x;
-            if (i < TP * groups) {
-                const int t = i / groups, G = i - t * groups;
+            if (tt[u] < TP) {
                 uint4 v = a[u];
                 if constexpr (!W4) {
                     uint32_t p[4];
                     permute_acts(a[u], p);
                     v = make_uint4(p[0], p[1], p[2], p[3]);
                 }
-                *reinterpret_cast<uint4*>(acts + t * S + act_slot(G) * 16) = v;
+                *reinterpret_cast<uint4*>(acts + tt[u] * S + act_slot(gg[u]) * 16) = v;
             }
         }
     }
@@ -155,11 +177,13 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
     }
     __syncthreads();
 
-    int acc[NT][4];
+    // The two MMAs of each word pair go to separate accumulators (no dependence between them);
+    // the sets are added after the loop.
+    int acc[NT][4], acc2[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
+        for (int i = 0; i < 4; ++i) acc[nt][i] = acc2[nt][i] = 0;
 
     for (int i0 = 0; i0 < my_n; i0 += PF) {
 #pragma unroll
@@ -181,7 +205,7 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
                         for (int nt = 0; nt < NT; ++nt) {
                             const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
                             mma_s8(acc[nt], a1, p.x, p.y);
-                            mma_s8(acc[nt], a2, p.z, p.w);
+                            mma_s8(acc2[nt], a2, p.z, p.w);
                         }
                     }
                     continue;
@@ -198,49 +222,45 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
                     for (int nt = 0; nt < NT; ++nt) {
                         const uint4 p = *reinterpret_cast<const uint4*>(acts + (nt * 8 + g) * S + slot * 16);
                         mma_s8(acc[nt], a1, p.x, p.y);
-                        mma_s8(acc[nt], a2, p.z, p.w);
+                        mma_s8(acc2[nt], a2, p.z, p.w);
                     }
                 }
             }
         }
     }
 
-    // Partial sums of this CTA's K slice: part[token][row] (row stride RBP: conflict-free).  With
-    // KSPLIT == 2 the odd-chunk warps write and the even-chunk warps of the same rows add theirs.
-    const int rl = rw * 16 + g;
-    if (ks == KSPLIT - 1) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] += acc2[nt][i];
+    // Each warp pushes its partial sums into the shared memory of the CTA that finishes its rows
+    // (distributed shared memory), into the slot of its source CTA and K parity, so one cluster
+    // barrier (release/acquire) suffices and no CTA reads another's memory after it.
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    {
+        const int rl = rw * 16 + g;                     // rl and rl + 8 have the same owner
+        const int owner = rl >> lg_rows, r0 = rl & (rows_per - 1);
+        int* dst = cluster.map_shared_rank(part, owner) + (rank * KSPLIT + ks) * TP * RPS;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int t0 = nt * 8 + 2 * qd;
-            part[t0 * RBP + rl] = acc[nt][0];
-            part[(t0 + 1) * RBP + rl] = acc[nt][1];
-            part[t0 * RBP + rl + 8] = acc[nt][2];
-            part[(t0 + 1) * RBP + rl + 8] = acc[nt][3];
-        }
-    }
-    if constexpr (KSPLIT == 2) __syncthreads();
-    if (KSPLIT == 2 && ks == 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int t0 = nt * 8 + 2 * qd;
-            part[t0 * RBP + rl] += acc[nt][0];
-            part[(t0 + 1) * RBP + rl] += acc[nt][1];
-            part[t0 * RBP + rl + 8] += acc[nt][2];
-            part[(t0 + 1) * RBP + rl + 8] += acc[nt][3];
+            if (QIFT_CK(owner < C && (t0 + 1) * RPS + r0 + 8 < TP * RPS)) {
+                dst[t0 * RPS + r0] = acc[nt][0];
+                dst[(t0 + 1) * RPS + r0] = acc[nt][1];
+                dst[t0 * RPS + r0 + 8] = acc[nt][2];
+                dst[(t0 + 1) * RPS + r0 + 8] = acc[nt][3];
+            }
         }
     }
     cluster.sync();
 
-    // CTA `rank` finishes rows [rank*RB/C, (rank+1)*RB/C) of the block: add the C partials;
-    // consecutive threads take consecutive rows of one token, so the stores run along n.
-    const int rows_per = RB / C;
+    // CTA `rank` finishes rows [rank*RB/C, (rank+1)*RB/C) of the block: add the received
+    // partials; consecutive threads take consecutive rows of one token, so the stores run along n.
 #pragma unroll 4
     for (int i = threadIdx.x; i < rows_per * TP; i += THREADS) {
-        const int t = i / rows_per, rl = rank * rows_per + (i - t * rows_per);
+        const int t = i >> lg_rows, r0 = i & (rows_per - 1), rl = rank * rows_per + r0;
         int sum = 0;
-        for (int p = 0; p < C; ++p)
-            if (QIFT_CK(p < (int)cluster.num_blocks() && t * RBP + rl < TP * RBP))
-                sum += cluster.map_shared_rank(part, p)[t * RBP + rl];
+        for (int sl = 0; sl < KSPLIT * C; ++sl) sum += part[(sl * TP + t) * RPS + r0];
         if constexpr (W4) sum >>= 4;  // exact: every product was 16 x level x q
         const int64_t n = (int64_t)row_block * RB + rl;
         if (t < T && n < N && QIFT_CK_RANGE((int64_t)t * N + n, 1, (int64_t)T * N)) {
@@ -248,7 +268,6 @@ __global__ void __launch_bounds__(32 * ROW_WARPS * KSPLIT) skinny_kernel(const i
             store_y<OutT>(y + (int64_t)t * N + n, v);
         }
     }
-    cluster.sync();  // keep this CTA's partials alive until every peer has read them
 }
 
 static int sm_count() {
@@ -265,7 +284,8 @@ static int sm_count() {
 template <int NT, int KSPLIT, bool W4, typename OutT>
 static cudaError_t launch_k(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
                             int64_t T, int64_t N, int64_t K, int C, int KS, OutT* y, cudaStream_t s) {
-    const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)NT * 8 * RBP * sizeof(int) + (size_t)(NT * 8 + RB) * 4;
+    const size_t smem = (size_t)NT * 8 * (KS + 64) + (size_t)KSPLIT * C * NT * 8 * (RB / C + 4) * sizeof(int) +
+                        (size_t)(NT * 8 + RB) * 4;
     cudaError_t e = ensure_smem(skinny_kernel<NT, KSPLIT, W4, OutT>, smem);
     if (e != cudaSuccess) return e;
     const int64_t blocks = (N + RB - 1) / RB;
