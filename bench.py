@@ -74,7 +74,7 @@ PROFILED_TRAFFIC = {
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
     "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="83bc35be637da8d0",
                     bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
-    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="fc3be88d2dbf2100", bytes=14853888 + 0,
+    "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="ff81329fc56d988a", bytes=14840320 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
     "offline": dict(files=("quantize_weights.cu", "common.cuh"), sha="00f7bc2d84fdc9a9",
                     bytes=67153920 + 1506816, scale=14336 * 4096 / (4096 * 4096),

@@ -310,14 +310,23 @@ static cudaError_t launch_k(const int8_t* q, const float* s_a, const uint32_t* c
 template <int NT, bool W4, typename OutT>
 static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* codes, const float* s_w, uint32_t lut,
                             int64_t T, int64_t N, int64_t K, OutT* y, cudaStream_t s) {
-    // Cluster size: split K so that each CTA streams a slice of at most 2048 inputs (64 KB of
-    // codes for its 128 rows) -- long-lived CTAs, yet enough of them when N is small.  C is a
-    // power of two <= 8, so it divides RB and every CTA finishes a whole number of rows.
+    // Cluster size C, a power of two <= 8 (so it divides RB): the smallest whose grid of
+    // blocks x C CTAs covers at least 80% of the SMs -- K is split, and partial sums reduced
+    // across the cluster, only as far as needed to fill the GPU -- and whose K slice of the
+    // activations fits shared memory.  Two warps share each 16-row group (16 warps per CTA)
+    // when the grid leaves an SM per CTA and the CTA has at least four K chunks; otherwise two
+    // 8-warp CTAs share an SM.  (A sweep of C and the warp split over the LLaMA shapes at 4-16
+    // tokens on B200 picked these within a few percent of the best for every shape.)
+    const int64_t blocks = (N + RB - 1) / RB;
+    const int sms = sm_count();
+    constexpr int CHUNK_K = CHUNK_WORDS * (W4 ? 8 : 16);
+    auto slice = [&](int c) { return (int)(((K + c - 1) / c + 255) / 256 * 256); };
     int C = 1;
-    while (C < 8 && (K + C - 1) / C > 2048) C *= 2;
-    const int KS = (int)(((K + C - 1) / C + 255) / 256 * 256);
-    const int64_t ctas = ((N + RB - 1) / RB) * C;
-    if (ctas <= sm_count()) return launch_k<NT, 2, W4, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
+    while (C < 8 && (blocks * C * 5 < (int64_t)sms * 4 || (size_t)NT * 8 * (slice(C) + 64) > 160 * 1024)) C *= 2;
+    const int KS = slice(C);
+    const int64_t ctas = blocks * C;
+    if (ctas <= sms && KS / CHUNK_K >= 4)
+        return launch_k<NT, 2, W4, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
     return launch_k<NT, 1, W4, OutT>(q, s_a, codes, s_w, lut, T, N, K, C, KS, y, s);
 }
 
