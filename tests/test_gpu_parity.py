@@ -552,6 +552,29 @@ def test_linear_each_kernel_family(path, name, T, N, K):
     assert qg.qift_device_error() == (qg.QIFT_OK, 0)
 
 
+@pytest.mark.parametrize("name", ["qift", "pot", "int4"])
+@pytest.mark.parametrize("T,N,K", [(16, 16000, 4096),   # 125 row blocks: no K split, two warps per row group
+                                   (16, 16000, 256),    # no K split, one chunk: one warp per row group
+                                   (8, 14336, 4096),    # clusters of 2, two CTAs per SM
+                                   (16, 4096, 4096),    # clusters of 4, one CTA per SM
+                                   (16, 1024, 4096),    # clusters of 8, two chunks per CTA
+                                   (3, 300, 14336)])    # clusters of 8, seven chunks per CTA
+def test_skinny_cluster_plans(name, T, N, K):
+    # The skinny kernel picks its cluster size (the K split) and its warps per row group from
+    # the grid it would launch; these shapes reach every cluster size and both warp splits.
+    qg.qift_debug_set_linear_path("skinny")
+    try:
+        for out_dtype in (torch.float16, torch.float32):
+            seed = 13 * T + N + K
+            got, ref = (_linear_w4_case(T, N, K, seed, out_dtype) if name == "int4"
+                        else _linear_case(name, T, N, K, seed, out_dtype))
+            u = np.uint16 if out_dtype == torch.float16 else np.uint32
+            assert np.array_equal(got.view(u), ref.view(u)), (name, T, N, K)
+    finally:
+        qg.qift_debug_set_linear_path("auto")
+    assert qg.qift_device_error() == (qg.QIFT_OK, 0)
+
+
 @pytest.mark.parametrize("name", ["qift", "pot"])
 @pytest.mark.parametrize("N,K", [(5, 64), (37, 1088), (300, 2112), (130, 4160), (64, 6208), (257, 11008), (3, 32768)])
 def test_linear_one_token_gemv_partial_chunks(name, N, K):
