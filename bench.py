@@ -1,16 +1,17 @@
 """Benchmark of the Qift W2A4 linear path on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|decode16|prefill|single|offline|decode_w4|decode16_w4]
+                    [--workload decode|decode16|prefill|single|offline|decode_w4|decode16_w4|prefill_w4]
 
 Workloads (synthetic, seeded; shapes of LLaMA linear modules):
   decode   (default) LLaMA-7B q_proj 4096x4096, 1 token, 4096-point Hadamard, Qift {+-1,+-3}
   decode16 LLaMA-3.1-8B MLP (gate/up 14336x4096, down 4096x14336), 16 tokens, 128-block, PoT
   prefill  LLaMA-7B MLP (gate/up 11008x4096, down 4096x11008), 2048 tokens, 128-block, Qift
   single   one 256x512 linear, 8 tokens (parity case; timed for completeness)
-  decode_w4, decode16_w4
-           the decode and decode16 shapes with 4-bit weights ({-7..7} * s per channel), the
-           W4 layers of a mixed W2/W4 model: W4A4 linear on CUDA cores
+  decode_w4, decode16_w4, prefill_w4
+           the decode, decode16 and prefill shapes with 4-bit weights ({-7..7} * s per channel),
+           the W4 layers of a mixed W2/W4 model: W4A4 linear (CUDA-core GEMV at one token, the
+           tensor-core skinny GEMM at 16, the tcgen05 pair GEMM at 2048)
   offline  offline quantization of a full 8B-shaped model (224 modules, 6.98 G weights):
            128-block rotation + per-row scale search + encode + pack for the Qift, PoT and
            standard level sets; reports weights/s and the reconstruction MSE of each set
@@ -105,7 +106,8 @@ def workload_def(name):
     from w2a4_gemm_b200 import synth
     return {"decode": synth.LLAMA7B_QPROJ_DECODE, "decode16": synth.LLAMA31_8B_MLP_DECODE16,
             "prefill": synth.LLAMA7B_MLP_PREFILL, "single": synth.SINGLE_256x512,
-            "decode_w4": synth.LLAMA7B_QPROJ_DECODE_W4, "decode16_w4": synth.LLAMA31_8B_MLP_DECODE16_W4}[name]
+            "decode_w4": synth.LLAMA7B_QPROJ_DECODE_W4, "decode16_w4": synth.LLAMA31_8B_MLP_DECODE16_W4,
+            "prefill_w4": synth.LLAMA7B_MLP_PREFILL_W4}[name]
 
 
 def code_bytes(N, K, levelset):
@@ -885,7 +887,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["decode", "decode16", "prefill", "single", "offline", "decode_w4",
-                                           "decode16_w4"], default="decode")
+                                           "decode16_w4", "prefill_w4"], default="decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-extra-stages", action="store_true",
                     help="decode workload only: skip the prefill and 16-token decode stages")

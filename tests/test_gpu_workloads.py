@@ -32,7 +32,8 @@ def host(t):
 
 CASES = [(wl.name, i) for wl in (synth.SINGLE_256x512, synth.LLAMA7B_QPROJ_DECODE, synth.LLAMA7B_MLP_PREFILL,
                                  synth.LLAMA31_8B_MLP_DECODE16, synth.LLAMA7B_QPROJ_DECODE_W4,
-                                 synth.LLAMA31_8B_MLP_DECODE16_W4) for i in range(len(wl.linears))]
+                                 synth.LLAMA31_8B_MLP_DECODE16_W4, synth.LLAMA7B_MLP_PREFILL_W4)
+         for i in range(len(wl.linears))]
 
 
 @pytest.mark.parametrize("wname,idx", CASES)

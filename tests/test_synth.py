@@ -54,6 +54,9 @@ def test_workload_shapes():
     assert (s.tokens, s.w_block, s.out_dtype, s.w_dist) == (8, 512, "f32", "normal")
     assert wl["llama7b_q_proj_decode_T1_w4"].levelset == "int4"
     assert wl["llama31_8b_mlp_decode_T16_w4"].levelset == "int4"
+    pw = wl["llama7b_mlp_prefill_T2048_w4"]
+    assert (pw.tokens, pw.w_block, pw.levelset) == (2048, 128, "int4")
+    assert [(l.n_out, l.n_in) for l in pw.linears] == [(l.n_out, l.n_in) for l in p.linears]
     # gate and up read the same input, down its own
     assert d.linears[0].x_seed == d.linears[1].x_seed != d.linears[2].x_seed
 

@@ -138,8 +138,20 @@ LLAMA31_8B_MLP_DECODE16_W4 = Workload(
              Linear("down_proj", 4096, 14336, (4, 2), (104, 2))),
 )
 
+LLAMA7B_MLP_PREFILL_W4 = Workload(
+    name="llama7b_mlp_prefill_T2048_w4",
+    description="LLaMA-7B MLP prefill: gate/up 11008x4096, down 4096x11008, 2048 tokens, "
+                "128-block Hadamard, 4-bit weights (W4A4)",
+    levelset="int4", w_block=128, a_block=128, tokens=2048, out_dtype="f16", w_dist="t4",
+    n_outliers=-1,
+    linears=(Linear("gate_proj", 11008, 4096, (3, 0), (103, 0)),
+             Linear("up_proj", 11008, 4096, (3, 1), (103, 0)),
+             Linear("down_proj", 4096, 11008, (3, 2), (103, 2))),
+)
+
 WORKLOADS = {w.name: w for w in (SINGLE_256x512, LLAMA7B_QPROJ_DECODE, LLAMA7B_MLP_PREFILL,
-                                 LLAMA31_8B_MLP_DECODE16, LLAMA7B_QPROJ_DECODE_W4, LLAMA31_8B_MLP_DECODE16_W4)}
+                                 LLAMA31_8B_MLP_DECODE16, LLAMA7B_QPROJ_DECODE_W4, LLAMA31_8B_MLP_DECODE16_W4,
+                                 LLAMA7B_MLP_PREFILL_W4)}
 
 # Offline quantization of a full 8B-shaped model: 32 layers x 7 linear modules.
 MODEL_8B_PROJS = (("q_proj", 4096, 4096), ("k_proj", 1024, 4096), ("v_proj", 1024, 4096),
