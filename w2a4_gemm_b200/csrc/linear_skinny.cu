@@ -8,12 +8,12 @@
 // Work split.  A thread-block cluster of C CTAs shares one block of 128 output rows; CTA r of
 // the cluster owns the K slice [r*KS, (r+1)*KS).  Each 16-row group of the block is owned by
 // one warp, or by two warps taking alternate 256-input chunks when the grid leaves an SM per
-// CTA (more warps in flight per SM).  The CTA
-// stages its slice of every token's int8 activations once in shared memory, permuted per
-// 16-byte group to the decode order, so the weights never touch shared memory: a lane loads
-// 16 bytes (4 words = 64 codes) of each of its two rows, decodes a word into four int8x4
-// registers with two masks, two shifts and four byte permutes against the level table, and
-// those registers ARE the A fragments of mma.m16n8k32 (s8 x s8 -> s32).  Each warp pushes its
+// CTA (more warps in flight per SM).  The CTA stages its slice of every token's int8
+// activations once in shared memory, permuted per 16-byte group to the decode order, so the
+// weights never touch shared memory: a lane loads 16 bytes (4 words = 64 codes) of each of its
+// two rows, decodes a word into four int8x4 registers with two masks, two shifts and four byte
+// permutes against the level table, and those registers ARE the A fragments of
+// mma.m16n8k32 (s8 x s8 -> s32).  Each warp pushes its
 // partial int32 sums into the shared memory of the cluster CTA that finishes those rows
 // (distributed shared memory); after one cluster barrier every CTA adds the partials it
 // received (exact, order-free) and finishes 128/C rows with the fp32 epilogue.  No global
