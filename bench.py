@@ -71,7 +71,7 @@ def peaks():
 # as null.  `scale` converts the captured launch to the benchmarked one when the shapes differ
 # (traffic grows in proportion to the weights processed).
 PROFILED_TRAFFIC = {
-    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="87eab3d8c0a24955", bytes=4225536 + 0,
+    "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="b4c3a19ee0236ba1", bytes=4226048 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
     "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="83bc35be637da8d0",
                     bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
