@@ -77,7 +77,7 @@ PROFILED_TRAFFIC = {
                     bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
     "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="4ec14ac10ad3f139", bytes=14840320 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
-    "decode_w4": dict(files=("linear_w4.cu", "common.cuh"), sha="e68c75357c803b87", bytes=8418816 + 0,
+    "decode_w4": dict(files=("linear_w4.cu", "common.cuh"), sha="bec1d0cc3845435a", bytes=8418560 + 0,
                       profile="profiles/w4_gemv1_kernel_q_proj_decode_T1_w4.md"),
     "decode16_w4": dict(files=("linear_skinny.cu", "common.cuh"), sha="4ec14ac10ad3f139", bytes=29514240 + 256,
                         profile="profiles/skinny_kernel_mlp_decode_T16_w4.md"),

@@ -26,7 +26,9 @@
 namespace qift {
 namespace w4 {
 
-constexpr int kWarps = 4;
+// Warps per CTA: 8 (256 CTAs at 4096 x 4096 for one token) measured 2.27 us per launch against
+// 2.32 us for 4.
+constexpr int kWarps = 8;
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(OutT* p, float v);
