@@ -18,6 +18,23 @@ def test_linear_bytes_q_proj_decode():
     assert bench.linear_bytes(1, 4096, 4096, 2, "int4") == 4096 * 4096 // 2 + 4 * 4096 + 4096 + 4 + 2 * 4096
 
 
+def test_traffic_records_match_the_current_kernels():
+    # Each DRAM-traffic record is keyed by a hash of its kernel's sources and reported as null once
+    # they change; every record on file must have been captured on the sources as they stand,
+    # next to its ncu summary.
+    for name, rec in bench.PROFILED_TRAFFIC.items():
+        assert bench.profiled_traffic(name) == rec["bytes"] * rec.get("scale", 1.0), name
+        assert os.path.exists(os.path.join(bench.ROOT, rec["profile"])), name
+    assert bench.profiled_traffic("single") is None  # no record: null, not a guess
+
+
+def test_every_workload_has_a_bench_choice():
+    from w2a4_gemm_b200 import synth
+    names = {bench.workload_def(w).name for w in ("decode", "decode16", "prefill", "single", "decode_w4",
+                                                     "decode16_w4", "prefill_w4")}
+    assert names == set(synth.WORKLOADS)
+
+
 def test_peaks_reads_measured_file_or_fallback():
     p = bench.peaks()
     assert p["hbm_gbs"] > 1000 and p["int8_tops"] > 1000
