@@ -73,8 +73,8 @@ def peaks():
 PROFILED_TRAFFIC = {
     "decode": dict(files=("linear_gemv.cu", "common.cuh"), sha="b4c3a19ee0236ba1", bytes=4226048 + 0,
                    profile="profiles/gemv1_kernel_q_proj_decode_T1.md"),
-    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="83bc35be637da8d0",
-                    bytes=19756544 + 3021312, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
+    "prefill": dict(files=("linear_gemm_tc.cu", "tc.cuh", "common.cuh"), sha="6f280e4dafa17a5e",
+                    bytes=19754752 + 2899456, profile="profiles/w2a4_gemm_pair_kernel_mlp_prefill_T2048.md"),
     "decode16": dict(files=("linear_skinny.cu", "common.cuh"), sha="4ec14ac10ad3f139", bytes=14840320 + 0,
                      profile="profiles/skinny_kernel_mlp_decode_T16_pot.md"),
     "decode_w4": dict(files=("linear_w4.cu", "common.cuh"), sha="bec1d0cc3845435a", bytes=8418560 + 0,

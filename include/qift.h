@@ -175,8 +175,9 @@ qift_status qift_dequantize_kv(const uint8_t* packed, const float* scales, int64
  * tensor-core GEMM, which needs n_in % 64 == 0: tokens >= 17 with another n_in returns
  * QIFT_ERR_UNSUPPORTED (pad n_in to a multiple of 64 with zero activations -- any code in the
  * padded positions then contributes nothing).  All paths give bit-identical results.
- * Overlap: the decode kernels are launched as programmatic dependents of the previous kernel
- * on `stream` and may start reading the weights -- `codes` and `w_scale`, nothing else --
+ * Overlap: every kernel of this call (decode sizes and the prefill GEMM) is launched as a
+ * programmatic dependent of the previous kernel on `stream` and may start reading the weights
+ * -- `codes` and `w_scale`, nothing else --
  * before that kernel has finished; the values of q_act and act_scale are read, and y written,
  * only after it has completed (their cache lines may be prefetched into L2 before, which
  * changes no value).  So the kernel launched immediately before qift_linear on the same stream

@@ -32,8 +32,9 @@ qift_status qift_debug_stall_next_gemm(void);
  * outputs, and qift_device_error() reports QIFT_ERR_TIMEOUT.  One-shot, per host thread. */
 qift_status qift_debug_stall_next_one_token(void);
 
-/* Turn programmatic dependent launch of the decode-size kernels on (default) or off, to
- * measure what the overlap with the previous kernel is worth.  Per host thread. */
+/* Turn programmatic dependent launch of the qift_linear and qift_decode_linear kernels on
+ * (default) or off, to measure what the overlap with the previous kernel is worth.  Per host
+ * thread. */
 qift_status qift_debug_set_pdl(int32_t enable);
 
 /* Pin the kernel family qift_linear uses: 0 = automatic (by batch size), 1 = CUDA-core GEMV

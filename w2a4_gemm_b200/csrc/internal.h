@@ -112,7 +112,7 @@ enum LinearPath {
 void debug_set_linear_path(int path);
 int debug_linear_path();
 void debug_set_pdl(bool on);
-bool pdl_enabled();  // programmatic dependent launch for the decode kernels (default on)
+bool pdl_enabled();  // programmatic dependent launch for the linear and decode kernels (default on)
 void debug_set_gemm_wait_limit(long long cycles);
 void debug_stall_next_gemm();
 

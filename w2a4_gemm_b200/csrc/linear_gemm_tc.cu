@@ -214,12 +214,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     tc::cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or copy
     tc::tc_fence_after();
+    // Programmatic dependent launch: the next kernel on the stream may be scheduled now; it
+    // waits for this grid's completion before it reads what this grid writes.
+    griddep_launch_dependents();
     const uint32_t tmem = *sm.tmem_base;
     volatile int* abort_v = reinterpret_cast<volatile int*>(sm.abort);
 
     if (warp == 0) {
         if (lane == 0) {  // ------------------------------------------------ TMA producer
             const uint32_t full0 = tc::cluster_addr(sm.full, 0);
+            // The codes of the first ring stages (weights: nothing a previous kernel on the stream
+            // writes) are requested before the wait for that kernel; the activations after it.
+            const int pre = total < STAGES ? total : STAGES;
+            for (int gp = 0; gp < pre; ++gp) {
+                const int ip = gp / num_kb, kbp = gp - ip * num_kb;
+                const Tile tp = tile_of(ip, pairs_x, rank);
+                const bool cod = tp.n0 < N;
+                tc::mbar_arrive_expect_tx(&sm.cfull[gp], cod ? COD_BYTES : 0);
+                if (cod && QIFT_CK(kbp * 16 * (W4 ? 8 : 16) < K && tp.n0 >= 0 && tp.n0 < N))
+                    tc::tma_load_2d(sm.cod + gp * COD_BYTES, &tmap_c, &sm.cfull[gp], kbp * 16, tp.n0);
+            }
+            griddep_wait();
             int g = 0;
             bool ok = true;
             for (int i = 0; ok && i < my_tiles; ++i) {
@@ -238,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     const bool second = !W4 && kb * BK + 128 < K;
                     if (rank == 0) tc::mbar_arrive_expect_tx(&sm.full[s], act_ctas * (second ? 2u : 1u) * ACT_HALF);
-                    tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
+                    if (g >= pre) tc::mbar_arrive_expect_tx(&sm.cfull[s], has_cod ? COD_BYTES : 0);
                     // tensor-map coordinates: x a 16-byte multiple inside the row, y inside the matrix
                     if (has_act && QIFT_CK((kb * BKI) % 16 == 0 && kb * BKI < K && tb >= 0 && tb < T)) {
                         tc::tma_load_2d_pair(sm.act + s * ACT_BYTES, &tmap_x, full0 + 8 * s, kb * BKI, tb);
@@ -246,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tc::tma_load_2d_pair(sm.act + s * ACT_BYTES + ACT_HALF, &tmap_x, full0 + 8 * s,
                                                  kb * BK + 128, tb);
                     }
-                    if (has_cod && QIFT_CK(kb * 16 * (W4 ? 8 : 16) < K && tl.n0 >= 0 && tl.n0 < N))
+                    if (g >= pre && has_cod && QIFT_CK(kb * 16 * (W4 ? 8 : 16) < K && tl.n0 >= 0 && tl.n0 < N))
                         tc::tma_load_2d(sm.cod + s * COD_BYTES, &tmap_c, &sm.cfull[s], kb * 16, tl.n0);
                 }
             }
@@ -379,6 +394,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         OutT* stg = reinterpret_cast<OutT*>(sm.stg);
         const bool vec_ok = ((int64_t)N * sizeof(OutT)) % 16 == 0;
         bool alive = true;
+        griddep_wait();  // the activation scales, and y, may belong to the previous kernel
         for (int i = 0; i < my_tiles; ++i) {
             const Tile tl = tile_of(i, pairs_x, rank);
             if (et < BNT) sm.sa[et] = tl.t0 + et < T ? s_a[tl.t0 + et] : 0.0f;
@@ -555,9 +571,18 @@ static cudaError_t launch_t(const int8_t* q, const float* s_a, const uint32_t* c
     const int clusters = (int)std::min<int64_t>(tiles, std::max(1, max_clusters<OutT, W4>()));
     const int stall = g_stall_next ? 1 : 0;
     g_stall_next = false;
-    w2a4_gemm_pair_kernel<OutT, W4><<<2 * clusters, kThreads, SMEM_BYTES, s>>>(mx, mc, s_a, s_w, lut, (int)T, (int)N,
-                                                                                (int)K, y, g_wait_limit, stall);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, w2a4_gemm_pair_kernel<OutT, W4>, mx, mc, s_a, s_w, lut, (int)T, (int)N, (int)K, y,
+                              g_wait_limit, stall);
 }
 
 }  // namespace gemm_pair
